@@ -1,0 +1,308 @@
+/*
+ * mqkv.h — C ABI of libmqkv, a B200 (sm_100a) library for a chunk-adaptive
+ * mixed-bitwidth KV cache.
+ *
+ * The library implements one data path, in three calls:
+ *
+ *   mq_route_chunks  a small router scores every context token against three
+ *                    quantisation "experts" {FP16, INT4, INT2}; each fixed-size
+ *                    chunk takes the majority choice of its tokens.
+ *                    (MoQAE paper notes, 方法详解 › 整体框架 and
+ *                     关键设计 › Quantization-Aware Experts.)
+ *   mq_build_layout  chunks of each sequence are regrouped by precision into
+ *                    contiguous FP16 → INT4 → INT2 segments before anything is
+ *                    quantised (Cocktail abstract on the "Bin Zhang" scholarfeed
+ *                    author page: chunk-level KV cache computation).
+ *   mq_pack_kv       K and V of one layer are quantised at the chunk's bitwidth
+ *                    and written into those segments.
+ *   mq_decode_attn   single-query attention for every sequence, read directly
+ *                    from the mixed-bitwidth packed cache.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers prefixed h_ are HOST memory; every other data pointer is DEVICE
+ *   memory on the current CUDA device.  All memory is owned by the caller; the
+ *   library never allocates, frees or retains a pointer after a call returns.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call that launches work is asynchronous on that stream and never
+ *   synchronises the host, except the two calls documented as synchronising
+ *   (mq_packed_bytes, mq_device_status).
+ * - Arguments are validated on the host before anything is launched.  A
+ *   failing check returns a non-zero mq_status, launches nothing, and leaves a
+ *   human-readable reason in mq_last_error() (thread-local).  Validation makes
+ *   no CUDA call, so it works on a machine without a GPU.
+ * - Device pointers must be 16-byte aligned.
+ * - Conditions that can only be seen on the device (for example a packed
+ *   buffer smaller than the layout needs) make the kernel skip its writes and
+ *   set a bit in a device-side status word, read with mq_device_status().
+ *
+ * Shapes and notation
+ * -------------------
+ *   B    = shape.num_seqs          sequences in the batch
+ *   Hq   = shape.num_q_heads       query heads
+ *   Hkv  = shape.num_kv_heads      key/value heads; Hq % Hkv == 0 (GQA when >1)
+ *   d    = shape.head_dim          64 or 128
+ *   L    = shape.chunk_len         tokens per routing chunk, a multiple of 32
+ *   G    = shape.group_size        quantisation group along head_dim, must be 32
+ *   T_b  = h_seq_lens[b]           tokens of sequence b (0 allowed)
+ *   n_b  = ceil(T_b / L)           chunks of sequence b; the last one may be short
+ *   T    = sum_b T_b,  N = sum_b n_b
+ *   expert / segment index s: 0 = FP16 (16 bits), 1 = INT4, 2 = INT2.
+ *
+ * d_cu_seqlens is a device int64[B+1] with d_cu_seqlens[0] = 0 and
+ * d_cu_seqlens[b+1] - d_cu_seqlens[b] = T_b: row r of C, K and V belongs to
+ * sequence b when d_cu_seqlens[b] <= r < d_cu_seqlens[b+1].
+ *
+ * Packed cache format (one buffer per layer; part of this ABI)
+ * ------------------------------------------------------------
+ * Per sequence b, segments in the order FP16, INT4, INT2.  A segment holds the
+ * sequence's chunks of that precision in their ORIGINAL chunk order (stable
+ * regrouping), so the short tail chunk, when present, is the last chunk of its
+ * segment.  Inside segment s of sequence b there are 2*Hkv regions, K regions
+ * for kv-heads 0..Hkv-1 first, then V regions 0..Hkv-1, each of
+ * layout.seq[b].region_bytes[s] bytes.  With n = seg_tokens[s] tokens:
+ *   FP16 region : codes = n rows of d IEEE binary16 values (2*d bytes a row),
+ *                 converted from the input with round-to-nearest-even (a copy
+ *                 for fp16 input); no scales.
+ *                 region_bytes = align128(n * 2*d).
+ *   INT-b region: codes  = n rows of d*b/8 bytes; group k (dims 32k..32k+31)
+ *                 fills bytes [4b*k, 4b*(k+1)) of the row.  Inside a group,
+ *                 element j sits at bit position b*(j mod (32/b)) of the
+ *                 little-endian 32-bit word j / (32/b) (least significant bits
+ *                 first).
+ *                 scales = n rows of d/32 pairs of binary16 (scale, min), the
+ *                 pair for group k at bytes [4k, 4k+4) of the row, scale in the
+ *                 low half.  They start at byte layout.seq[b].scale_offset[s]
+ *                 = align128(n * d*b/8) of the region.
+ *                 region_bytes = scale_offset + align128(n * (d/32) * 4).
+ *   Row i of a region is segment token i: token t of the chunk at reordered
+ *   position p sits at row (p - seg_chunk_begin[s]) * L + t.
+ *   Segment s of sequence b starts at byte layout.seq[b].seg_base[s]; bases
+ *   are consecutive in (b, s) order (each segment is 2*Hkv*region_bytes long,
+ *   a multiple of 128), and the buffer is layout.header.packed_bytes long.
+ *   Padding bytes are unspecified.
+ *
+ * Quantiser (spec reading; the MoQAE notes leave it open)
+ * --------------------------------------------------------------
+ * For every (token, kv-head, group of 32) of an INT-b chunk, with x the fp32
+ * value of each element (fp16 input widened exactly):
+ *   mn = min x, mx = max x                                  (fp32)
+ *   s  = (mx - mn) / (2^b - 1)   IEEE fp32 subtract and divide, s = 1 if mx == mn
+ *   q  = min(max(rint((x - mn) / s), 0), 2^b - 1)   fp32 subtract and divide,
+ *        rint rounds half to even, no FMA contraction, no fast-math
+ *   stored: q bit-packed, (half)s and (half)mn rounded to nearest even.
+ * Inputs must be finite with |x| < 65504 (undefined otherwise).
+ * Dequantised value: xhat = q * (half)s + (half)mn.
+ */
+#ifndef MQKV_H_
+#define MQKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mq_status {
+  MQ_OK = 0,
+  MQ_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape */
+  MQ_ERR_UNSUPPORTED = 2,   /* valid in principle, not built (e.g. d = 96) */
+  MQ_ERR_WORKSPACE = 3,     /* caller buffer smaller than the call needs */
+  MQ_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  MQ_ERR_DEVICE_CHECK = 5   /* a kernel reported a failed check */
+} mq_status;
+
+typedef enum mq_dtype {
+  MQ_F32 = 0,               /* IEEE binary32 */
+  MQ_F16 = 1                /* IEEE binary16 */
+} mq_dtype;
+
+typedef enum mq_expert {
+  MQ_EXPERT_FP16 = 0,
+  MQ_EXPERT_INT4 = 1,
+  MQ_EXPERT_INT2 = 2
+} mq_expert;
+
+typedef struct mq_shape {
+  int32_t num_seqs;      /* B   >= 1 */
+  int32_t num_q_heads;   /* Hq  >= 1 */
+  int32_t num_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0, Hq / Hkv <= 8 */
+  int32_t head_dim;      /* d: 64 or 128 */
+  int32_t chunk_len;     /* L: multiple of 32, 32 <= L <= 4096 */
+  int32_t group_size;    /* G: must be 32 */
+} mq_shape;
+
+/* Device-side status bits (mq_device_status). */
+#define MQ_DEV_PACKED_TOO_SMALL   0x1u  /* packed_bytes < layout packed size */
+#define MQ_DEV_WORKSPACE_TOO_SMALL 0x2u /* decode schedule exceeds workspace */
+#define MQ_DEV_BAD_LAYOUT         0x4u  /* layout magic/shape mismatch */
+#define MQ_DEV_WAIT_TIMEOUT       0x8u  /* a bounded wait on a copy gave up */
+#define MQ_DEV_INDEX_RANGE        0x10u /* an index left its valid range */
+
+/* ---------------------------------------------------------------------------
+ * Layout table (device memory written by mq_build_layout; part of this ABI).
+ *
+ *   [mq_layout_header][mq_seq_layout x B][int32 perm[N] (padded to 16 B)]
+ *   [int32 inv[N] (padded to 16 B)]
+ *
+ * perm[chunk_offset_b + p] = original chunk index of the chunk stored at
+ * reordered position p of sequence b; inv is its inverse (original index ->
+ * reordered position); both are local to the sequence.
+ * Fields marked "schedule" describe how mq_decode_attn splits the work; they
+ * are implementation-defined (any split that covers every segment token once
+ * is valid) and are not part of the method.
+ * ------------------------------------------------------------------------- */
+#define MQ_LAYOUT_MAGIC 0x4C4B514Du   /* "MQKL" */
+#define MQ_LAYOUT_VERSION 1u
+
+typedef struct mq_layout_header {
+  uint32_t magic;           /* MQ_LAYOUT_MAGIC */
+  uint32_t version;         /* MQ_LAYOUT_VERSION */
+  int32_t  num_seqs;        /* B */
+  int32_t  num_kv_heads;    /* Hkv */
+  int32_t  head_dim;        /* d */
+  int32_t  chunk_len;       /* L */
+  int32_t  total_chunks;    /* N */
+  int32_t  total_items;     /* schedule: work items per kv-head */
+  int64_t  total_tokens;    /* T */
+  uint64_t packed_bytes;    /* bytes of one layer's packed buffer */
+  int32_t  item_tokens[3];  /* schedule: max tokens of a work item, per segment */
+  int32_t  reserved[1];     /* zero */
+} mq_layout_header;         /* 64 bytes */
+
+typedef struct mq_seq_layout {
+  int64_t  token_offset;      /* d_cu_seqlens[b] */
+  int32_t  num_tokens;        /* T_b */
+  int32_t  num_chunks;        /* n_b */
+  int32_t  chunk_offset;      /* sum of n_b' for b' < b */
+  int32_t  seg_chunks[3];     /* chunks in each segment */
+  int32_t  seg_chunk_begin[3];/* first reordered position of each segment */
+  int32_t  seg_tokens[3];     /* tokens in each segment */
+  uint64_t seg_base[3];       /* byte offset of each segment in packed */
+  uint64_t region_bytes[3];   /* bytes of one (K|V, kv-head) region */
+  uint64_t scale_offset[3];   /* byte offset of scales inside an INT region (0 for FP16) */
+  int32_t  item_begin[3];     /* schedule: first work item of (b, s) */
+  int32_t  item_count[3];     /* schedule: work items of (b, s) */
+  int32_t  reserved[2];       /* zero */
+} mq_seq_layout;              /* 160 bytes */
+
+/* ---------------------------------------------------------------------------
+ * Status and sizes
+ * ------------------------------------------------------------------------- */
+
+/* Static text for a status code. Never NULL. */
+const char* mq_status_string(mq_status status);
+
+/* Reason for the last failing call on this thread ("" if none). */
+const char* mq_last_error(void);
+
+/* Bytes of the layout table for this shape and these lengths; 0 if the
+ * arguments are invalid (see mq_last_error). */
+size_t mq_layout_bytes(const mq_shape* shape, const int32_t* h_seq_lens);
+
+/* Bytes of one layer's packed buffer if every chunk were FP16 — an upper bound
+ * for any routing map. 0 if the arguments are invalid. */
+size_t mq_packed_bytes_upper_bound(const mq_shape* shape, const int32_t* h_seq_lens);
+
+/* Bytes of workspace mq_decode_attn needs for a layout built from this shape
+ * and these lengths. 0 if the arguments are invalid. */
+size_t mq_decode_workspace_bytes(const mq_shape* shape, const int32_t* h_seq_lens);
+
+/* Reads layout.header.packed_bytes into *h_bytes. SYNCHRONISES `stream`. */
+mq_status mq_packed_bytes(const void* layout, size_t* h_bytes, void* stream);
+
+/* Synchronises `stream`, then stores the device status word (MQ_DEV_* bits,
+ * OR-ed over every kernel since the last clear) in *h_flags; clears it when
+ * `clear` is non-zero. Returns MQ_ERR_DEVICE_CHECK when any bit is set. */
+mq_status mq_device_status(uint32_t* h_flags, int32_t clear, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_route_chunks — router, per-token argmax, per-chunk vote, routing freezing.
+ *
+ * MoQAE paper notes, 关键设计 › Quantization-Aware Experts: the router maps a
+ * chunk C (rows = tokens, D features) to one score per expert for every token,
+ * printed as f(CW1·CW2)W3.  This library reads that as the gated MLP
+ *     z_t = (SiLU(C_t W1) ⊙ (C_t W2)) W3 + b3,   SiLU(x) = x / (1 + e^-x)
+ * evaluated in fp32.  Every token picks argmax_e z_t[e] (an exact tie goes to
+ * the lower index = more bits); every chunk takes the expert most of its
+ * tokens picked (a tie in counts goes to the lower index).  With
+ * routing_freeze != 0, chunk 0 of every sequence is forced to FP16
+ * (路由冻结 / Routing Freezing).  The map is computed once per sequence from
+ * the router input C; the caller reuses the resulting layout for every layer
+ * (路由共享 / Routing Sharing).
+ *
+ *   C            device fp32 [T, D] row-major (row r = token r, see d_cu_seqlens)
+ *   W1, W2       device fp32 [D, H] row-major
+ *   W3           device fp32 [H, 3] row-major
+ *   b3           device fp32 [3], or NULL for zero bias
+ *   token_expert device uint8 [T]  out: per-token argmax
+ *   chunk_expert device uint8 [N]  out: per-chunk expert, chunk (b, c) at
+ *                                  index chunk_offset_b + c
+ *   logits       device fp32 [T, 3] out, or NULL
+ * Constraints: 1 <= D, D % 4 == 0; H in {64, 128, 256}.
+ * ------------------------------------------------------------------------- */
+mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
+                          const int64_t* d_cu_seqlens,
+                          const float* C, int32_t D, int32_t H,
+                          const float* W1, const float* W2, const float* W3,
+                          const float* b3, int32_t routing_freeze,
+                          uint8_t* token_expert, uint8_t* chunk_expert,
+                          float* logits, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_build_layout — Cocktail's chunk regrouping (chunk-level KV cache
+ * computation): stable partition of each sequence's chunks by precision into
+ * FP16 → INT4 → INT2 segments, with perm/inv tables, segment token counts and
+ * byte offsets of the packed format above.
+ *
+ *   chunk_expert device uint8 [N], values 0..2 (other values: treated as INT2
+ *                and MQ_DEV_INDEX_RANGE is set)
+ *   layout       device buffer of at least mq_layout_bytes(shape, h_seq_lens)
+ * One layout serves every layer (routing sharing) and every decode step.
+ * ------------------------------------------------------------------------- */
+mq_status mq_build_layout(const mq_shape* shape, const int32_t* h_seq_lens,
+                          const int64_t* d_cu_seqlens,
+                          const uint8_t* chunk_expert,
+                          void* layout, size_t layout_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_pack_kv — quantise one layer's K and V at each chunk's bitwidth (the
+ * quantiser above) and write them into the packed format.
+ *
+ *   K, V         device [T, Hkv, d] row-major, dtype kv_dtype (MQ_F16 or MQ_F32)
+ *   packed       device buffer of packed_bytes bytes; must be at least the
+ *                layout's packed_bytes (checked on the device: if it is
+ *                smaller nothing is written and MQ_DEV_PACKED_TOO_SMALL is set)
+ * ------------------------------------------------------------------------- */
+mq_status mq_pack_kv(const mq_shape* shape, const int32_t* h_seq_lens,
+                     const void* layout, const void* K, const void* V,
+                     int32_t kv_dtype, void* packed, size_t packed_bytes,
+                     void* stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_decode_attn — one decode query per (sequence, query head) attends over
+ * every cached token of its sequence (MoQAE notes, 整体框架: ordinary attention
+ * after quantisation), reading the packed cache directly:
+ *   o[b,h] = sum_t softmax_t(scale * q[b,h] · khat_t) vhat_t
+ * with khat/vhat the dequantised K/V of kv-head h / (Hq/Hkv).  Work is split
+ * into precision-homogeneous pieces of one segment each; a second pass merges
+ * the pieces' (max, sum, accumulator) triples.
+ *
+ *   q            device [B, Hq, d], dtype q_dtype (MQ_F16 or MQ_F32)
+ *   softmax_scale  <= 0 selects 1/sqrt(d)
+ *   out          device fp32 [B, Hq, d]; a sequence with T_b = 0 gets zeros
+ *   workspace    device buffer of at least mq_decode_workspace_bytes(shape,
+ *                h_seq_lens) bytes; contents on entry are ignored
+ * ------------------------------------------------------------------------- */
+mq_status mq_decode_attn(const mq_shape* shape, const int32_t* h_seq_lens,
+                         const void* layout, const void* packed,
+                         const void* q, int32_t q_dtype, float softmax_scale,
+                         float* out, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MQKV_H_ */
