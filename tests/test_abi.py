@@ -1,0 +1,139 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+function include/mqkv.h declares, validates arguments before touching CUDA,
+and its size queries agree with the header's closed forms (checked through
+the CPU oracle's independent implementation of the format)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from chunk_adaptive_mixed_b200 import build as B
+from chunk_adaptive_mixed_b200 import mqkv as M
+from oracle import oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "mqkv.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+    yield
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mq_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(M.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(M.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for st in range(6):
+        assert M.status_string(st)
+    assert M.status_string(99) == "unknown status"
+
+
+def _shape(**kw):
+    base = dict(num_seqs=2, num_q_heads=8, num_kv_heads=2, head_dim=128, chunk_len=64)
+    base.update(kw)
+    return M.shape(**base)
+
+
+LENS = np.array([300, 64], np.int32)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_seqs=0), M.MQ_ERR_INVALID_ARG),
+    (dict(num_q_heads=6, num_kv_heads=4), M.MQ_ERR_INVALID_ARG),
+    (dict(num_q_heads=12, num_kv_heads=4), M.MQ_ERR_UNSUPPORTED),   # Hq/Hkv = 3
+    (dict(head_dim=96), M.MQ_ERR_UNSUPPORTED),
+    (dict(chunk_len=48), M.MQ_ERR_INVALID_ARG),
+    (dict(chunk_len=16), M.MQ_ERR_INVALID_ARG),
+    (dict(group_size=64), M.MQ_ERR_UNSUPPORTED),
+])
+def test_bad_shapes_are_rejected_before_any_launch(kw, status):
+    lib = M.lib()
+    shp = _shape(**kw)
+    lens = np.array([300, 64], np.int32)
+    dummy = 1 << 20  # aligned, never dereferenced
+    st = lib.mq_pack_kv(ctypes.byref(shp), lens.ctypes.data, dummy, dummy, dummy, M.MQ_F16, dummy,
+                        1 << 20, 0)
+    assert st == status, M.last_error()
+    assert M.last_error()
+    assert lib.mq_layout_bytes(ctypes.byref(shp), lens.ctypes.data) == 0
+
+
+def test_bad_pointers_and_sizes():
+    lib = M.lib()
+    shp = _shape()
+    lens = LENS.copy()
+    p = 1 << 20
+    # null / misaligned device pointers
+    assert lib.mq_pack_kv(ctypes.byref(shp), lens.ctypes.data, None, p, p, 1, p, 1 << 20, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    assert "layout" in M.last_error()
+    assert lib.mq_pack_kv(ctypes.byref(shp), lens.ctypes.data, p + 4, p, p, 1, p, 1 << 20, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    assert "aligned" in M.last_error()
+    # negative length
+    bad = np.array([300, -1], np.int32)
+    assert lib.mq_pack_kv(ctypes.byref(shp), bad.ctypes.data, p, p, p, 1, p, 1 << 20, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    # wrong dtype code
+    assert lib.mq_pack_kv(ctypes.byref(shp), lens.ctypes.data, p, p, p, 7, p, 1 << 20, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    # router: H unsupported, D not a multiple of 4
+    assert lib.mq_route_chunks(ctypes.byref(shp), lens.ctypes.data, p, p, 64, 96, p, p, p, None, 1,
+                               p, p, None, 0) == M.MQ_ERR_UNSUPPORTED
+    assert lib.mq_route_chunks(ctypes.byref(shp), lens.ctypes.data, p, p, 66, 64, p, p, p, None, 1,
+                               p, p, None, 0) == M.MQ_ERR_INVALID_ARG
+    # layout buffer too small
+    need = lib.mq_layout_bytes(ctypes.byref(shp), lens.ctypes.data)
+    assert lib.mq_build_layout(ctypes.byref(shp), lens.ctypes.data, p, p, p, need - 16, 0) \
+        == M.MQ_ERR_WORKSPACE
+    # decode workspace too small
+    ws = lib.mq_decode_workspace_bytes(ctypes.byref(shp), lens.ctypes.data)
+    assert ws > 0
+    assert lib.mq_decode_attn(ctypes.byref(shp), lens.ctypes.data, p, p, p, 1, 0.0, p, p, ws - 1,
+                              0) == M.MQ_ERR_WORKSPACE
+    assert lib.mq_packed_bytes(None, None, 0) == M.MQ_ERR_INVALID_ARG
+    assert lib.mq_device_status(None, 0, 0) == M.MQ_ERR_INVALID_ARG
+
+
+def test_valid_call_without_gpu_reports_cuda_error():
+    # no silent CPU path: with valid arguments and no device the call fails
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    lib = M.lib()
+    shp = _shape()
+    lens = LENS.copy()
+    p = 1 << 20
+    need = lib.mq_layout_bytes(ctypes.byref(shp), lens.ctypes.data)
+    st = lib.mq_build_layout(ctypes.byref(shp), lens.ctypes.data, p, p, p, need, 0)
+    assert st == M.MQ_ERR_CUDA, M.last_error()
+
+
+@pytest.mark.parametrize("d,L", [(64, 32), (128, 64), (128, 256)])
+def test_size_queries_match_the_format(d, L):
+    rng = np.random.default_rng(d + L)
+    lens = rng.integers(0, 2000, 5).astype(np.int32)
+    shp = _shape(num_seqs=5, head_dim=d, chunk_len=L)
+    n = int(((lens + L - 1) // L).sum())
+    assert M.mq_layout_bytes(shp, lens) == O.layout_bytes(lens, L)
+    assert M.mq_packed_bytes_upper_bound(shp, lens) == \
+        O.packed_bytes(2, d, L, lens, np.zeros(n, np.uint8))
+    ce = rng.integers(0, 3, n).astype(np.uint8)
+    assert O.packed_bytes(2, d, L, lens, ce) <= M.mq_packed_bytes_upper_bound(shp, lens)
