@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the chunk-adaptive mixed-bitwidth KV-cache path on B200.
+
+One step = one pass of the whole path over one batch:
+  route (router scores, argmax, vote, freezing)  ->  layout (regroup by
+  precision)  ->  pack every layer  ->  one decode step per layer,
+all through the C ABI of libmqkv, on synthetic inputs already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle, timed as a baseline
+
+Default workload: llama2_7b_32l (Llama-2-7B shape, 32 layers sharing one
+routing map, 4 x 32768 tokens, chunk 128).  Multi-GPU (torchrun): every rank
+runs its own batch (seeded by rank), no data-path collective; the timed
+region is bracketed by barriers and the max over ranks is reported.
+
+Printed: one JSON line on rank 0.  value = decode tokens per second of the
+whole step (sequences x decode steps / step time, summed over ranks).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attn tokens/s & packed-KV HBM GB/s (% of B200 peak); pack GB/s"
+DEFAULT_WORKLOAD = "llama2_7b_32l"
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our path
+
+class Setup:
+    """Device-resident inputs and outputs of one batch of the workload."""
+
+    def __init__(self, w, seed, device):
+        import torch
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        from chunk_adaptive_mixed_b200 import workloads as W
+        self.w = w
+        self.lens = W.seq_lens(w, seed)
+        self.B = len(self.lens)
+        self.T = int(self.lens.sum())
+        self.N = int(W.num_chunks(self.lens, w.chunk_len).sum())
+        self.shape = M.shape(self.B, w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_len)
+        self.cu = torch.as_tensor(W.cu_seqlens(self.lens), device=device)
+        self.W1, self.W2, self.W3, self.b3 = W.router_weights(w, seed, device)
+        self.C = W.router_input(w, self.lens, seed, device)
+        self.K, self.V, self.q = [], [], []
+        for layer in range(w.layers):
+            K, V = W.kv_layer(w, self.lens, layer, seed, device)
+            self.K.append(K)
+            self.V.append(V)
+            self.q.append([W.query(w, layer, s, seed, device) for s in range(w.decode_steps)])
+        u8 = torch.uint8
+        self.token_expert = torch.empty(self.T, dtype=u8, device=device)
+        self.chunk_expert = torch.empty(max(self.N, 16), dtype=u8, device=device)
+        self.layout = torch.empty(M.mq_layout_bytes(self.shape, self.lens), dtype=u8,
+                                  device=device)
+        # packed buffers sized for any routing map (all-FP16 bound): no host
+        # round trip is needed between routing and packing
+        ub = M.mq_packed_bytes_upper_bound(self.shape, self.lens)
+        self.packed = [torch.empty(ub, dtype=u8, device=device) for _ in range(w.layers)]
+        self.out = [torch.empty(self.B, w.num_q_heads, w.head_dim, dtype=torch.float32,
+                                device=device) for _ in range(w.layers)]
+        self.ws = torch.empty(M.mq_decode_workspace_bytes(self.shape, self.lens), dtype=u8,
+                              device=device)
+        self.kv_bytes = sum(K.numel() * K.element_size() * 2 for K in self.K) // w.layers
+        torch.cuda.synchronize()
+
+    def step(self, timers=None):
+        """One pass of the whole path (launches only; asynchronous)."""
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        w = self.w
+        M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, self.W1, self.W2, self.W3,
+                          self.b3, self.token_expert, self.chunk_expert)
+        M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_expert, self.layout)
+        for layer in range(w.layers):
+            if timers:
+                timers["pack"][layer][0].record()
+            M.mq_pack_kv(self.shape, self.lens, self.layout, self.K[layer], self.V[layer],
+                         self.packed[layer])
+            if timers:
+                timers["pack"][layer][1].record()
+        for s in range(w.decode_steps):
+            for layer in range(w.layers):
+                if timers and s == 0:
+                    timers["decode"][layer][0].record()
+                M.mq_decode_attn(self.shape, self.lens, self.layout, self.packed[layer],
+                                 self.q[layer][s], self.out[layer], self.ws)
+                if timers and s == 0:
+                    timers["decode"][layer][1].record()
+
+    def launches_per_step(self):
+        # router + vote, 2 layout kernels, one pack per layer, two decode
+        # kernels per layer and decode step
+        return 2 + 2 + self.w.layers + 2 * self.w.layers * self.w.decode_steps
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from chunk_adaptive_mixed_b200 import build as Bld
+    from chunk_adaptive_mixed_b200 import mqkv as M
+    from chunk_adaptive_mixed_b200 import workloads as W
+    Bld.build()
+    M.lib()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    w = W.get(args.workload)
+    seed = args.seed + 1009 * rank
+    S = Setup(w, seed, device)
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    for _ in range(args.warmup):
+        S.step()
+    torch.cuda.synchronize()
+    assert M.mq_device_status() == 0, "device-side check failed during warm-up"
+    pb = M.mq_packed_bytes(S.layout)
+    mix = np.bincount(S.chunk_expert[:S.N].cpu().numpy(), minlength=3) / max(S.N, 1)
+
+    # per-kernel events for every pack launch and the first decode step
+    E = torch.cuda.Event
+    timers_all = []
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    t_start, t_end = E(enable_timing=True), E(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        tm = {"pack": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)],
+              "decode": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)]}
+        S.step(tm)
+        timers_all.append(tm)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    assert M.mq_device_status() == 0, "device-side check failed in the timed region"
+    ms = t_start.elapsed_time(t_end)
+    if dist:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    pack_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["pack"]]
+    dec_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["decode"]]
+    pack_avg = float(np.mean(pack_ms))
+    dec_avg = float(np.mean(dec_ms))
+
+    tokens_per_step = S.B * w.decode_steps
+    value = tokens_per_step * world / (ms_step / 1e3)
+    peak, peak_kind = measured_peaks()
+    pack_bytes = S.kv_bytes + pb                                   # read K/V, write packed
+    dec_bytes = pb + sum(x.numel() * x.element_size() for x in (S.q[0][0], S.out[0]))
+    pack_gbs = pack_bytes / (pack_avg / 1e3) / 1e9
+    dec_gbs = dec_bytes / (dec_avg / 1e3) / 1e9
+
+    # end to end through the same calls, inputs in pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(S, args, device)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, S.lens, seed, tokens_per_step)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; random tensors of the model's shape, no checkpoint)",
+            "config": {"workload": w.name, "layers": w.layers, "num_seqs": S.B,
+                       "seq_len": int(S.lens.max()), "total_tokens": S.T,
+                       "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
+                       "head_dim": w.head_dim, "chunk_len": w.chunk_len,
+                       "router_D": w.router_dim, "router_H": w.router_hidden,
+                       "kv_dtype": w.kv_dtype, "decode_steps": w.decode_steps,
+                       "parallelism": f"dp{world} (independent batches)",
+                       "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
+                       else "inputs fit in L2"},
+            "roofline": {"bound": "hbm", "kernel": "pack_kernel",
+                         "achieved": pack_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": pack_gbs / peak, "traffic": None,
+                         "peak_source": peak_kind,
+                         "algorithmic_bytes_per_launch": pack_bytes,
+                         "avg_launch_ms": pack_avg},
+            "decode_attn": {"GB/s": dec_gbs, "frac": dec_gbs / peak, "avg_ms_per_layer": dec_avg,
+                            "tokens_per_s_attention_only": S.B / (dec_avg * w.layers / 1e3),
+                            "algorithmic_bytes_per_layer": dec_bytes},
+            "pack": {"GB/s": pack_gbs, "frac": pack_gbs / peak, "avg_ms_per_layer": pack_avg},
+            "packed_bytes_per_layer": pb,
+            "chunk_mix": [round(float(x), 4) for x in mix],
+            "avg_bits": float(np.dot(mix, [16, 4, 2])),
+            "clocks": clocks,
+            "gpu_launches": S.launches_per_step() * args.steps,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(S, args, device):
+    """Same step through the same ABI calls, with every step's inputs copied
+    from pinned host memory inside the timed region and each layer's output
+    read back."""
+    import torch
+    w = S.w
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    host = {}
+    host["C"] = pinned_copy(S.C)
+    host["K"] = [pinned_copy(K) for K in S.K]
+    host["V"] = [pinned_copy(V) for V in S.V]
+    host["q"] = [[pinned_copy(q) for q in qs] for qs in S.q]
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in S.out]
+    h2d = (host["C"].numel() * 4 + sum(x.numel() * x.element_size() for x in host["K"] + host["V"])
+           + sum(q.numel() * q.element_size() for qs in host["q"] for q in qs))
+    d2h = sum(o.numel() * o.element_size() for o in out_host) * w.decode_steps
+
+    def e2e_step():
+        S.C.copy_(host["C"], non_blocking=True)
+        for layer in range(w.layers):
+            S.K[layer].copy_(host["K"][layer], non_blocking=True)
+            S.V[layer].copy_(host["V"][layer], non_blocking=True)
+            for s in range(w.decode_steps):
+                S.q[layer][s].copy_(host["q"][layer][s], non_blocking=True)
+        S.step()
+        for layer in range(w.layers):
+            out_host[layer].copy_(S.out[layer], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    E = torch.cuda.Event
+    a, b = E(enable_timing=True), E(enable_timing=True)
+    a.record()
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.e2e_steps
+    del host
+    return {"value": S.B * w.decode_steps / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": args.e2e_steps,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_step_estimate(w, lens, seed, route_chunks=32, pack_tokens=32768):
+    """Times the CPU oracle on a bounded sample of one step and scales each
+    phase to the full step.  Returns (seconds per full step, sample text, cores)."""
+    import torch
+    from chunk_adaptive_mixed_b200 import workloads as W
+    from oracle import oracle as O
+    L = w.chunk_len
+    W1, W2, W3, b3 = (x.numpy() for x in W.router_weights(w, seed, "cpu"))
+    T = int(lens.sum())
+    N = int(W.num_chunks(lens, L).sum())
+    # routing: the first route_chunks chunks
+    nr = min(route_chunks, N)
+    C = W.router_input(w, lens, seed, "cpu", chunk_range=(0, nr)).numpy()
+    counts = W.chunk_token_counts(lens, L)[:nr].astype(np.int32)
+    t0 = time.perf_counter()
+    z32, _ = O.router_logits(C, W1, W2, W3, b3)
+    O.vote(counts, L, O.token_argmax(z32), True)
+    t_route = (time.perf_counter() - t0) * T / max(int(counts.sum()), 1)
+    # packing and decode: 1 layer of the first sequence, capped at pack_tokens
+    Tp = int(min(lens[0], pack_tokens))
+    lens1 = np.array([Tp], np.int32)
+    K, V = W.kv_layer(w, lens1, 0, seed, "cpu")
+    cmap = W.synthetic_chunk_map(lens1, L, mix=w.target_mix, seed=1)
+    Kn, Vn = K.numpy(), V.numpy()
+    t0 = time.perf_counter()
+    packed = O.pack(w.num_kv_heads, w.head_dim, L, lens1, cmap, Kn, Vn)
+    t_pack = (time.perf_counter() - t0) * (T / Tp) * w.layers
+    # decode: 1 layer of the same sample
+    q = W.query(w, 0, 0, seed, "cpu").numpy()[:1]
+    t0 = time.perf_counter()
+    O.decode(w.num_q_heads, w.num_kv_heads, w.head_dim, L, lens1, cmap, packed, q)
+    t_dec = (time.perf_counter() - t0) * (T / Tp) * w.layers * w.decode_steps
+    sample = (f"route {int(counts.sum())} tokens, pack + decode {Tp} tokens of 1 layer; "
+              f"each phase scaled to {T} tokens x {w.layers} layers x {w.decode_steps} "
+              f"decode step(s)")
+    return t_route + t_pack + t_dec, sample, O.num_threads()
+
+
+def cpu_baseline(w, lens, seed, tokens_per_step):
+    t, sample, cores = oracle_step_estimate(w, lens, seed)
+    return {"value": tokens_per_step / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": sample, "projected_s_per_step": t}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on bounded samples."""
+    if rank != 0:
+        return
+    from chunk_adaptive_mixed_b200 import workloads as W
+    w = W.get(args.workload)
+    lens = W.seq_lens(w, args.seed)
+    tokens_per_step = len(lens) * w.decode_steps
+    # a smaller sample per step than the cpu_baseline leg, so that K + W
+    # steps stay within a few minutes
+    kw = dict(route_chunks=8, pack_tokens=8192)
+    for _ in range(args.warmup):
+        oracle_step_estimate(w, lens, args.seed, **kw)
+    times = []
+    t_start = time.perf_counter()
+    for _ in range(args.steps):
+        t, sample, cores = oracle_step_estimate(w, lens, args.seed, **kw)
+        times.append(t)
+    wall = time.perf_counter() - t_start
+    t_step = float(np.mean(times))
+    value = tokens_per_step / t_step
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "layers": w.layers, "num_seqs": len(lens),
+                       "total_tokens": int(lens.sum()), "parallelism": "rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "sample_wall_s": wall}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus > 1 and world == 1:
+        raise SystemExit("--gpus > 1 needs torchrun (one process per GPU)")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
