@@ -107,6 +107,14 @@ mq_status check_lens(const mq_shape* s, const int32_t* h_seq_lens, int64_t* T, i
 
 }  // namespace
 
+mq_status report_error(mq_status status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+  return status;
+}
+
 // ------------------------------------------------------------ item policy
 
 ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens) {

@@ -119,6 +119,9 @@ cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layo
                           float* out, void* workspace, size_t workspace_bytes,
                           unsigned int* status, cudaStream_t stream);
 
+// Records a formatted reason for mq_last_error() and returns `status`.
+mq_status report_error(mq_status status, const char* fmt, ...);
+
 // Workspace layout of mq_decode_attn for a given item bound.
 size_t decode_workspace_bytes(const mq_shape& s, int64_t max_items);
 

@@ -36,7 +36,10 @@ MQ_DEV_INDEX_RANGE = 0x10
 # names of every function include/mqkv.h declares
 EXPORTS = ("mq_status_string", "mq_last_error", "mq_layout_bytes", "mq_packed_bytes_upper_bound",
            "mq_decode_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
-           "mq_build_layout", "mq_pack_kv", "mq_decode_attn")
+           "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc")
+
+# size of the scratch array built into the library for mq_decode_attn_noalloc
+MQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class MqShape(ctypes.Structure):
@@ -89,6 +92,8 @@ def lib() -> ctypes.CDLL:
     L.mq_pack_kv.argtypes = [sp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.mq_decode_attn.restype = ctypes.c_int
     L.mq_decode_attn.argtypes = [sp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp, sz, vp]
+    L.mq_decode_attn_noalloc.restype = ctypes.c_int
+    L.mq_decode_attn_noalloc.argtypes = [sp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp]
     _lib = L
     return L
 
@@ -213,3 +218,13 @@ def mq_decode_attn(shp, seq_lens, layout, packed, q, out, workspace, softmax_sca
     _check(lib().mq_decode_attn(ctypes.byref(shp), l.ctypes.data, _ptr(layout), _ptr(packed),
                                 _ptr(q), _dtype_code(q), float(softmax_scale), _ptr(out),
                                 _ptr(workspace), nbytes, _stream(stream)), "mq_decode_attn")
+
+
+def mq_decode_attn_noalloc(shp, seq_lens, layout, packed, q, out, softmax_scale=0.0, stream=None):
+    """mq_decode_attn using the library's built-in scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    l = _lens(seq_lens)
+    _check(lib().mq_decode_attn_noalloc(ctypes.byref(shp), l.ctypes.data, _ptr(layout),
+                                        _ptr(packed), _ptr(q), _dtype_code(q),
+                                        float(softmax_scale), _ptr(out), _stream(stream)),
+           "mq_decode_attn_noalloc")

@@ -301,6 +301,38 @@ mq_status mq_decode_attn(const mq_shape* shape, const int32_t* h_seq_lens,
                          float* out, void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/* ---------------------------------------------------------------------------
+ * mq_decode_attn_noalloc — mq_decode_attn without a caller workspace.
+ *
+ * The paper has no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: for example a serving runtime that reserves
+ * nearly all of HBM for its own KV pool at start-up and permits no later
+ * cudaMalloc, or a plain C host program with no device allocator of its own.
+ * The per-item partial results go to a scratch array of
+ * MQ_NOALLOC_SCRATCH_BYTES bytes that is part of the library's module image:
+ * every GPU that loads the library holds it until the process exits.
+ *
+ *   Arguments: as mq_decode_attn, without workspace / workspace_bytes.
+ *   Limit: fails with MQ_ERR_WORKSPACE, before anything is launched, when
+ *          mq_decode_workspace_bytes(shape, h_seq_lens) exceeds
+ *          MQ_NOALLOC_SCRATCH_BYTES; otherwise errors as mq_decode_attn.
+ *   Set-up: the first call on each device looks up the array's device
+ *          address (cudaGetSymbolAddress) with that device current; make that
+ *          first call before any stream capture begins.
+ *   Sharing: every call uses the same array, which keeps what the last call
+ *          wrote.  Calls whose work overlaps on the GPU (other streams, other
+ *          host threads) race on it and corrupt each other's results.
+ *          Nothing in it has to start at zero: each entry the merge pass
+ *          reads is written earlier in the same call.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * ------------------------------------------------------------------------- */
+#define MQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+mq_status mq_decode_attn_noalloc(const mq_shape* shape, const int32_t* h_seq_lens,
+                                 const void* layout, const void* packed,
+                                 const void* q, int32_t q_dtype, float softmax_scale,
+                                 float* out, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif
