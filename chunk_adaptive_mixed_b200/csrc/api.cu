@@ -118,28 +118,29 @@ mq_status report_error(mq_status status, const char* fmt, ...) {
 // ------------------------------------------------------------ item policy
 
 ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens) {
-  // The largest item of each precision fills at most 32 KiB of staging (K+V
-  // codes and scales) and QPG * tokens <= 2048 scores; smaller problems are
-  // split finer (by powers of two, down to 32 tokens) so that there are at
-  // least ~8 items per SM of a 148-SM part.  Depends only on the shape and
-  // the lengths, so size queries and layout builds agree without a GPU.
+  // A work item carries about 32 KiB of packed K+V (64 KiB when four or more
+  // query heads share a kv-head, whose per-item partial results are larger),
+  // so the partial results stay a few percent of the bytes read.  Small
+  // problems are split finer (by powers of two, down to 32 tokens) so that
+  // there are at least ~8 items per SM of a 148-SM part.  Depends only on the
+  // shape and the lengths, so size queries and layout builds agree without a
+  // GPU.
   const int d = s.head_dim;
   const int qpg = s.num_q_heads / s.num_kv_heads;
   const int bpt[kNumExperts] = {2 * 2 * d, 2 * (d / 2 + d / 8), 2 * (d / 4 + d / 8)};
-  int cap_scores = (2048 / qpg) / 32 * 32;
+  const int target = 32768 * (qpg >= 4 ? 2 : 1);
   ItemPolicy p;
   for (int e = 0; e < kNumExperts; ++e) {
-    int m = (32768 / bpt[e]) / 32 * 32;
-    if (m > cap_scores) m = cap_scores;
+    int m = (target / bpt[e]) / 32 * 32;
     if (m < 32) m = 32;
     p.item_tokens[e] = m;
   }
   int64_t T = 0;
   for (int b = 0; b < s.num_seqs; ++b) T += h_seq_lens[b];
-  const int64_t target = 148 * 8;
+  const int64_t want = 148 * 8;
   while (true) {
     const int64_t est = T * s.num_kv_heads / p.item_tokens[1];
-    if (est >= target) break;
+    if (est >= want) break;
     bool shrunk = false;
     for (int e = 0; e < kNumExperts; ++e)
       if (p.item_tokens[e] >= 64) {

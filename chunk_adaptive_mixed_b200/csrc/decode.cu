@@ -29,71 +29,48 @@
 namespace mqkv {
 namespace {
 
-constexpr int kDecThreads = 128;
-constexpr int kStageBytes = 32768;
-constexpr int kMaxScores = 2048;  // QPG * tokens of one item
-constexpr int kMaxQpg = 8;
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr int kDecWarps = 8;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kRing = 4;  // stages of each warp's copy ring
 
-struct DecodeSmem {
-  alignas(128) unsigned char stage[kStageBytes + 64];
-  alignas(16) float q[kMaxQpg][4][36];  // [head][group][dim], rows padded
-  float qsum[kMaxQpg][4];
-  float sc[kMaxScores];  // scores, then probabilities, [head][token]
-  float m[kMaxQpg];
-  float l[kMaxQpg];
-  alignas(8) unsigned long long bar;
-  int info[8];  // b, s, n, g, kc_off, ks_off, vc_off, vs_off (stage offsets)
-  int abort_flag;
+// Lane geometry of one precision: each lane owns SL consecutive dims of one
+// token (SL * QPG query values and accumulators stay in registers), LPT lanes
+// cover a token, TPW tokens are processed per warp iteration.
+template <int D, int QPG, int E>
+struct Geo {
+  static constexpr int BITS = E == 0 ? 16 : (E == 1 ? 4 : 2);
+  static constexpr int SL_INT = 32 / QPG;
+  static constexpr int SL = E == 0 ? (SL_INT < 8 ? SL_INT : 8) : SL_INT;
+  static constexpr int LPT = D / SL;
+  static constexpr int TPW = 32 / LPT;
+  static constexpr int PIECE = SL * BITS / 8;   // code bytes of one lane's slice
+  static constexpr int CROW = D * BITS / 8;     // code bytes of one token row
+  static constexpr int SROW = E == 0 ? 0 : D / kGroup * 4;
+  static constexpr int CODES = TPW * CROW;      // code bytes of one iteration (K or V)
+  static constexpr int SCALES = E == 0 ? 0 : (TPW * SROW + 15) / 16 * 16;
+  static constexpr int STAGE = 2 * CODES + 2 * SCALES;
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+template <int D, int QPG>
+constexpr int stage_bytes() {
+  constexpr int a = Geo<D, QPG, 0>::STAGE, b = Geo<D, QPG, 1>::STAGE, c = Geo<D, QPG, 2>::STAGE;
+  constexpr int m = a > b ? a : b;
+  return (m > c ? m : c + 0) + 0;
 }
 
-__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+template <int D, int QPG>
+constexpr size_t decode_smem_bytes() {
+  return (size_t)kDecWarps * kRing * stage_bytes<D, QPG>();
 }
 
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
 }
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
-                                              unsigned long long* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait; returns false when the limit was reached.
-__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // exact small integer -> float: the integer is OR-ed into the mantissa of
@@ -108,7 +85,353 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t bits) {
   return __half22float2(h);
 }
 
-template <int D>
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic, round to nearest)
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+}
+__device__ __forceinline__ uint64_t pk2u(uint32_t a, uint32_t b) {
+  return (uint64_t)a | ((uint64_t)b << 32);
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Code extraction without shifts.  __byte_perm puts byte m of a code word
+// into bytes 2 and 1 of a word whose byte 3 is 0x43 (the exponent of 2^7):
+//   [0x43 | B | B | 0].
+// Masking keeps one code in the mantissa, giving exactly 128 + c * 2^k:
+//   INT4: low nibble  & 0xFF0F0000 -> 128 + c        (k = 0)
+//         high nibble & 0xFF00F000 -> 128 + c / 16   (k = -4, from byte 1)
+//   INT2: & 0xFF030000 -> 128 + c, & 0xFF0C0000 -> 128 + 4c,
+//         & 0xFF300000 -> 128 + 16c, & 0xFF00C000 -> 128 + c / 4.
+// (Byte 2's top bit is the exponent's lowest bit, so the code in that
+// position is read from the byte-1 copy instead.)  Each value has at most 12
+// significant bits, so its product with an fp16 query (11 bits), pre-scaled
+// by 2^-k, is exact in fp32.
+__device__ __forceinline__ uint32_t spread_byte(uint32_t word, int m) {
+  return __byte_perm(word, 0x43u, 0x4005u | ((uint32_t)m << 8) | ((uint32_t)m << 4));
+}
+
+// Per-position scale 2^-k of the code values above (query pre-scaling), and
+// its inverse (applied to value accumulators at the end).
+template <int BITS>
+__device__ __forceinline__ constexpr float pos_scale(int i) {
+  if constexpr (BITS == 4) return i % 2 == 0 ? 1.0f : 16.0f;
+  else return (i % 4) == 0 ? 1.0f : ((i % 4) == 1 ? 0.25f : ((i % 4) == 2 ? 0.0625f : 4.0f));
+}
+
+// One lane's copy units of one iteration: 16-byte pieces of the iteration's
+// token tile (K codes | V codes | K scales | V scales), located once per item.
+template <int STAGE>
+struct CopyPlan {
+  static constexpr int U = (STAGE / 16 + 31) / 32;
+  const unsigned char* src[U];  // source at iteration 0
+  uint32_t step[U];             // source advance per iteration
+  uint16_t dst[U];              // offset inside a stage
+  int16_t row[U];               // first token row (inside the tile) the unit reads
+  bool used[U];
+};
+
+template <typename Gm, int STAGE>
+__device__ __forceinline__ void plan_copies(CopyPlan<STAGE>& cp, const unsigned char* regk,
+                                            const unsigned char* regv, uint64_t soff, int64_t t0) {
+  const int lane = threadIdx.x & 31;
+  constexpr int CB = Gm::CODES, SB = Gm::SCALES;
+  constexpr int UNITS = (2 * CB + 2 * SB) / 16;
+#pragma unroll
+  for (int i = 0; i < CopyPlan<STAGE>::U; ++i) {
+    const int u = lane + 32 * i;
+    cp.used[i] = u < UNITS;
+    int off = u * 16;
+    if (off < CB) {
+      cp.src[i] = regk + t0 * Gm::CROW + off;
+      cp.step[i] = Gm::TPW * Gm::CROW;
+      cp.dst[i] = off;
+      cp.row[i] = off / Gm::CROW;
+    } else if ((off -= CB) < CB) {
+      cp.src[i] = regv + t0 * Gm::CROW + off;
+      cp.step[i] = Gm::TPW * Gm::CROW;
+      cp.dst[i] = CB + off;
+      cp.row[i] = off / Gm::CROW;
+    } else if ((off -= CB) < SB) {
+      cp.src[i] = regk + soff + t0 * Gm::SROW + off;
+      cp.step[i] = Gm::TPW * Gm::SROW;
+      cp.dst[i] = 2 * CB + off;
+      cp.row[i] = off / (Gm::SROW > 0 ? Gm::SROW : 1);
+    } else {
+      off -= SB;
+      cp.src[i] = regv + soff + t0 * Gm::SROW + off;
+      cp.step[i] = Gm::TPW * Gm::SROW;
+      cp.dst[i] = 2 * CB + SB + off;
+      cp.row[i] = off / (Gm::SROW > 0 ? Gm::SROW : 1);
+    }
+  }
+}
+
+template <int D, int QPG, int QDT, int E>
+__device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
+                                         const unsigned char* __restrict__ regv, uint64_t soff,
+                                         int t0, int n, const void* __restrict__ q, int64_t qbase,
+                                         float scale_log2, unsigned char* ring, int64_t w,
+                                         float* __restrict__ ws_acc, float2* __restrict__ ws_ml) {
+  using Gm = Geo<D, QPG, E>;
+  constexpr int SL = Gm::SL, LPT = Gm::LPT, TPW = Gm::TPW;
+  constexpr int STRIDE = stage_bytes<D, QPG>();
+  constexpr int BITS = Gm::BITS;
+  constexpr int NP = SL / 2;  // value pairs per lane
+  const int lane = threadIdx.x & 31;
+  const int tl = lane / LPT, sl = lane % LPT;
+  const int iters = (n + TPW - 1) / TPW;
+
+  CopyPlan<STRIDE> cp;
+  plan_copies<Gm, STRIDE>(cp, regk, regv, soff, t0);
+  auto issue = [&](int it) {
+    if (it < iters) {
+      const int nv = min(TPW, n - it * TPW);
+      unsigned char* st = ring + (it % kRing) * STRIDE;
+#pragma unroll
+      for (int i = 0; i < CopyPlan<STRIDE>::U; ++i)
+        if (cp.used[i] && cp.row[i] < nv)
+          cp_async16(st + cp.dst[i], cp.src[i] + (uint64_t)it * cp.step[i]);
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int it = 0; it < kRing - 1; ++it) issue(it);
+
+  // ---- query slice of every head, in value pairs, pre-scaled per code position
+  uint64_t qp[QPG][NP];
+  float qs[QPG], qb[QPG];
+#pragma unroll
+  for (int h = 0; h < QPG; ++h) {
+    const int64_t base = qbase + (int64_t)h * D + sl * SL;
+    qs[h] = 0.f;
+    qb[h] = 0.f;
+#pragma unroll
+    for (int j = 0; j < SL; j += 2) {
+      float a, b;
+      if constexpr (QDT == MQ_F16) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(static_cast<const __half*>(q) + base + j));
+        a = f.x;
+        b = f.y;
+      } else {
+        const float2 f = *reinterpret_cast<const float2*>(static_cast<const float*>(q) + base + j);
+        a = f.x;
+        b = f.y;
+      }
+      qs[h] += a + b;
+      if constexpr (E != 0) {
+        a *= pos_scale<BITS>(j);
+        b *= pos_scale<BITS>(j + 1);
+        qb[h] += a + b;
+      }
+      qp[h][j / 2] = pk2(a, b);
+    }
+    qb[h] *= 128.0f;
+  }
+
+  uint64_t acc[QPG][NP];
+  float bias[QPG], m[QPG], l[QPG];
+#pragma unroll
+  for (int h = 0; h < QPG; ++h) {
+    bias[h] = 0.f;
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) acc[h][j] = 0ull;
+  }
+  const uint64_t k128 = pk2(128.0f, 128.0f);
+  const int grp = (sl * SL) / kGroup;
+
+  for (int it = 0; it < iters; ++it) {
+    issue(it + kRing - 1);
+    cp_async_wait<kRing - 1>();
+    __syncwarp();
+    const unsigned char* st = ring + (it % kRing) * STRIDE;
+    const bool valid = it * TPW + tl < n;
+    const unsigned char* kp = st + tl * Gm::CROW + sl * Gm::PIECE;
+    const unsigned char* vp = st + Gm::CODES + tl * Gm::CROW + sl * Gm::PIECE;
+    float ks = 1.f, km = 0.f, vs = 1.f, vm = 0.f;
+    if constexpr (E != 0) {
+      const float2 a = half2_bits_to_float2(
+          *reinterpret_cast<const uint32_t*>(st + 2 * Gm::CODES + tl * Gm::SROW + grp * 4));
+      const float2 b = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(
+          st + 2 * Gm::CODES + Gm::SCALES + tl * Gm::SROW + grp * 4));
+      ks = a.x; km = a.y; vs = b.x; vm = b.y;
+    }
+    // ---- scores: q . code (pairs), then the group's scale and min
+    uint64_t dot2[QPG];
+#pragma unroll
+    for (int h = 0; h < QPG; ++h) dot2[h] = 0ull;
+    if constexpr (E == 0) {
+      const uint32_t* wv = reinterpret_cast<const uint32_t*>(kp);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const float2 f = half2_bits_to_float2(wv[i]);
+        const uint64_t x = pk2(f.x, f.y);
+#pragma unroll
+        for (int h = 0; h < QPG; ++h) dot2[h] = fma2(x, qp[h][i], dot2[h]);
+      }
+    } else {
+      constexpr int BYTES = SL * BITS / 8;
+      uint32_t words[(BYTES + 3) / 4];
+      if constexpr (BYTES >= 4) {
+#pragma unroll
+        for (int k = 0; k < BYTES / 4; ++k) words[k] = reinterpret_cast<const uint32_t*>(kp)[k];
+      } else {
+        words[0] = BYTES == 2 ? *reinterpret_cast<const unsigned short*>(kp) : *kp;
+      }
+#pragma unroll
+      for (int mb = 0; mb < BYTES; ++mb) {
+        const uint32_t t = spread_byte(words[mb / 4], mb % 4);
+        if constexpr (BITS == 4) {
+          const uint64_t x = pk2u(t & 0xFF0F0000u, t & 0xFF00F000u);
+#pragma unroll
+          for (int h = 0; h < QPG; ++h) dot2[h] = fma2(x, qp[h][mb], dot2[h]);
+        } else {
+          const uint64_t x0 = pk2u(t & 0xFF030000u, t & 0xFF0C0000u);
+          const uint64_t x1 = pk2u(t & 0xFF300000u, t & 0xFF00C000u);
+#pragma unroll
+          for (int h = 0; h < QPG; ++h) {
+            dot2[h] = fma2(x0, qp[h][2 * mb], dot2[h]);
+            dot2[h] = fma2(x1, qp[h][2 * mb + 1], dot2[h]);
+          }
+        }
+      }
+    }
+    float part[QPG];
+#pragma unroll
+    for (int h = 0; h < QPG; ++h) {
+      const float dot = lo2(dot2[h]) + hi2(dot2[h]);
+      part[h] = E == 0 ? dot : fmaf(ks, dot - qb[h], km * qs[h]);
+    }
+#pragma unroll
+    for (int off = 1; off < LPT; off <<= 1)
+#pragma unroll
+      for (int h = 0; h < QPG; ++h) part[h] += __shfl_xor_sync(0xffffffffu, part[h], off);
+    float p[QPG];
+#pragma unroll
+    for (int h = 0; h < QPG; ++h) {
+      const float sc = valid ? part[h] * scale_log2 : -INFINITY;
+      if (sc > m[h]) {  // new running maximum: rescale what was accumulated
+        const float a = exp2f(m[h] - sc);
+        const uint64_t a2 = pk2(a, a);
+        l[h] *= a;
+        bias[h] *= a;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) acc[h][j] = fma2(acc[h][j], a2, 0ull);
+        m[h] = sc;
+      }
+      p[h] = valid ? exp2f(sc - m[h]) : 0.f;
+      l[h] += p[h];
+    }
+    // ---- values (lanes past the item's last token hold stale stage bytes,
+    // which may decode to NaN: they skip the accumulation instead)
+    if (valid) {
+      uint64_t w2[QPG];
+#pragma unroll
+      for (int h = 0; h < QPG; ++h) {
+        const float wgt = E == 0 ? p[h] : p[h] * vs;
+        w2[h] = pk2(wgt, wgt);
+        if constexpr (E != 0) bias[h] = fmaf(p[h], vm, bias[h]);
+      }
+      if constexpr (E == 0) {
+        const uint32_t* wv = reinterpret_cast<const uint32_t*>(vp);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          const float2 f = half2_bits_to_float2(wv[i]);
+          const uint64_t x = pk2(f.x, f.y);
+#pragma unroll
+          for (int h = 0; h < QPG; ++h) acc[h][i] = fma2(x, w2[h], acc[h][i]);
+        }
+      } else {
+        constexpr int BYTES = SL * BITS / 8;
+        uint32_t words[(BYTES + 3) / 4];
+        if constexpr (BYTES >= 4) {
+#pragma unroll
+          for (int k = 0; k < BYTES / 4; ++k) words[k] = reinterpret_cast<const uint32_t*>(vp)[k];
+        } else {
+          words[0] = BYTES == 2 ? *reinterpret_cast<const unsigned short*>(vp) : *vp;
+        }
+#pragma unroll
+        for (int mb = 0; mb < BYTES; ++mb) {
+          const uint32_t t = spread_byte(words[mb / 4], mb % 4);
+          if constexpr (BITS == 4) {
+            const uint64_t x = sub2(pk2u(t & 0xFF0F0000u, t & 0xFF00F000u), k128);
+#pragma unroll
+            for (int h = 0; h < QPG; ++h) acc[h][mb] = fma2(x, w2[h], acc[h][mb]);
+          } else {
+            const uint64_t x0 = sub2(pk2u(t & 0xFF030000u, t & 0xFF0C0000u), k128);
+            const uint64_t x1 = sub2(pk2u(t & 0xFF300000u, t & 0xFF00C000u), k128);
+#pragma unroll
+            for (int h = 0; h < QPG; ++h) {
+              acc[h][2 * mb] = fma2(x0, w2[h], acc[h][2 * mb]);
+              acc[h][2 * mb + 1] = fma2(x1, w2[h], acc[h][2 * mb + 1]);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();  // every lane is done with this stage before it is refilled
+  }
+  cp_async_wait<0>();
+
+  // ---- undo the per-position code scaling, then merge the TPW token lanes
+  float av[QPG][SL];
+#pragma unroll
+  for (int h = 0; h < QPG; ++h)
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      av[h][2 * j] = lo2(acc[h][j]) * (E == 0 ? 1.f : pos_scale<BITS>(2 * j));
+      av[h][2 * j + 1] = hi2(acc[h][j]) * (E == 0 ? 1.f : pos_scale<BITS>(2 * j + 1));
+    }
+#pragma unroll
+  for (int off = LPT; off < 32; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < QPG; ++h) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[h], off);
+      const float bo = __shfl_xor_sync(0xffffffffu, bias[h], off);
+      const float M = fmaxf(m[h], mo);
+      const float a = m[h] == -INFINITY ? 0.f : exp2f(m[h] - M);
+      const float b = mo == -INFINITY ? 0.f : exp2f(mo - M);
+      l[h] = l[h] * a + lo * b;
+      bias[h] = bias[h] * a + bo * b;
+#pragma unroll
+      for (int j = 0; j < SL; ++j) {
+        const float ao = __shfl_xor_sync(0xffffffffu, av[h][j], off);
+        av[h][j] = av[h][j] * a + ao * b;
+      }
+      m[h] = M;
+    }
+  }
+  if (tl == 0) {
+#pragma unroll
+    for (int h = 0; h < QPG; ++h) {
+      float* dst = ws_acc + ((size_t)w * QPG + h) * D + sl * SL;
+#pragma unroll
+      for (int j = 0; j < SL; j += 4)
+        *reinterpret_cast<float4*>(dst + j) =
+            make_float4(av[h][j] + bias[h], av[h][j + 1] + bias[h], av[h][j + 2] + bias[h],
+                        av[h][j + 3] + bias[h]);
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < QPG; ++h) ws_ml[(size_t)w * QPG + h] = make_float2(m[h], l[h]);
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ int find_item_seq(const unsigned char* layout, int B, int64_t bs) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
@@ -120,354 +443,121 @@ __device__ __forceinline__ int find_item_seq(const unsigned char* layout, int B,
   return lo;
 }
 
+// Each warp is an independent worker: it takes work items w = warp id,
+// warp id + total warps, ... and streams each through its own copy ring.  No
+// block-wide barrier is used.
 template <int D, int QPG, int QDT>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, 2)
 decode_partial_kernel(const unsigned char* __restrict__ layout,
                       const unsigned char* __restrict__ packed, const void* __restrict__ q,
                       float scale_log2, float* __restrict__ ws_acc, float2* __restrict__ ws_ml,
                       int64_t capacity_items, unsigned int* status) {
-  constexpr int G = D / kGroup;
-  constexpr int S = D / 8;                 // 8-dim slices
-  constexpr int TL = kDecThreads / S;      // token lanes in the value pass
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
-
   const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
   if (h->magic != MQ_LAYOUT_MAGIC || h->head_dim != D) {
     if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_BAD_LAYOUT);
     return;
   }
-  const int B = h->num_seqs, Hkv = h->num_kv_heads, L = h->chunk_len;
-  (void)L;
+  const int B = h->num_seqs, Hkv = h->num_kv_heads;
   const int64_t total = (int64_t)h->total_items * Hkv;
   if (total > capacity_items) {
     if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_WORKSPACE_TOO_SMALL);
     return;
   }
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    mbar_init(&sm.bar, 1);
-    fence_barrier_init();
-    sm.abort_flag = 0;
-  }
-  __syncthreads();
-  uint32_t parity = 0;
-
-  for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
-    if (tid == 0) {
-      const int64_t bs = w / Hkv;
-      const int g = (int)(w - bs * Hkv);
-      const int b = find_item_seq<D>(layout, B, bs);
-      const mq_seq_layout* r =
-          reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
-      const int s = bs < r->item_begin[1] ? 0 : (bs < r->item_begin[2] ? 1 : 2);
-      const int j = (int)(bs - r->item_begin[s]);
-      const int it = h->item_tokens[s];
-      const int t0 = j * it;
-      const int n = min(it, r->seg_tokens[s] - t0);
-      const uint32_t crow = code_row_bytes(D, s);
-      const unsigned char* regk = packed + r->seg_base[s] + (uint64_t)g * r->region_bytes[s];
-      const unsigned char* regv = regk + (uint64_t)Hkv * r->region_bytes[s];
-      const uint32_t cbytes = (uint32_t)align16((uint64_t)n * crow);
-      const uint32_t sbytes = s == 0 ? 0u : (uint32_t)align16((uint64_t)n * scale_row_bytes(D));
-      const int kc = 0, ks = (int)cbytes, vc = (int)(cbytes + sbytes), vs = (int)(2 * cbytes + sbytes);
-      if (n <= 0 || n * QPG > kMaxScores || 2 * (cbytes + sbytes) > (uint32_t)kStageBytes) {
-        set_status(status, MQ_DEV_INDEX_RANGE);
-        sm.info[2] = 0;
-      } else {
-        sm.info[2] = n;
-      }
-      sm.info[0] = b; sm.info[1] = s; sm.info[3] = g;
-      sm.info[4] = kc; sm.info[5] = ks; sm.info[6] = vc; sm.info[7] = vs;
-      if (sm.info[2] > 0) {
-        fence_proxy_async_smem();
-        mbar_expect_tx(&sm.bar, 2 * (cbytes + sbytes));
-        bulk_copy_g2s(sm.stage + kc, regk + (uint64_t)t0 * crow, cbytes, &sm.bar);
-        bulk_copy_g2s(sm.stage + vc, regv + (uint64_t)t0 * crow, cbytes, &sm.bar);
-        if (s != 0) {
-          const uint32_t srow = scale_row_bytes(D);
-          bulk_copy_g2s(sm.stage + ks, regk + r->scale_offset[s] + (uint64_t)t0 * srow, sbytes,
-                        &sm.bar);
-          bulk_copy_g2s(sm.stage + vs, regv + r->scale_offset[s] + (uint64_t)t0 * srow, sbytes,
-                        &sm.bar);
-        }
-      }
-    }
-    __syncthreads();
-    const int b = sm.info[0], s = sm.info[1], n = sm.info[2], g = sm.info[3];
-    if (n == 0) {
-      __syncthreads();
+  const int warp = threadIdx.x / 32;
+  unsigned char* ring = smem_raw + (size_t)warp * kRing * stage_bytes<D, QPG>();
+  const int64_t nwarps = (int64_t)gridDim.x * kDecWarps;
+  for (int64_t w = (int64_t)blockIdx.x * kDecWarps + warp; w < total; w += nwarps) {
+    const int64_t bs = w / Hkv;
+    const int g = (int)(w - bs * Hkv);
+    const int b = find_item_seq(layout, B, bs);
+    const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
+    const int s = bs < r->item_begin[1] ? 0 : (bs < r->item_begin[2] ? 1 : 2);
+    const int j = (int)(bs - r->item_begin[s]);
+    const int t0 = j * h->item_tokens[s];
+    const int n = min(h->item_tokens[s], r->seg_tokens[s] - t0);
+    if (n <= 0) {
+      if ((threadIdx.x & 31) == 0) set_status(status, MQ_DEV_INDEX_RANGE);
       continue;
     }
-
-    // query heads of this kv-head, as fp32, while the copy is in flight
-    const int64_t qbase = ((int64_t)b * Hkv * QPG + (int64_t)g * QPG) * D;
-    for (int i = tid; i < QPG * D; i += kDecThreads) {
-      const int hh = i / D, dd = i - hh * D;
-      float v;
-      if constexpr (QDT == MQ_F16)
-        v = __half2float(static_cast<const __half*>(q)[qbase + i]);
-      else
-        v = static_cast<const float*>(q)[qbase + i];
-      sm.q[hh][dd / kGroup][dd % kGroup] = v;
-    }
-    __syncthreads();
-    if (tid < QPG * G) {
-      const int hh = tid / G, k = tid % G;
-      float acc = 0.f;
-#pragma unroll
-      for (int j = 0; j < kGroup; ++j) acc += sm.q[hh][k][j];
-      sm.qsum[hh][k] = acc;
-    }
-
-    bool ok = mbar_wait_bounded(&sm.bar, parity);
-    parity ^= 1u;
-    if (!ok) {
-      set_status(status, MQ_DEV_WAIT_TIMEOUT);
-      atomicExch(&sm.abort_flag, 1);
-      mbar_wait_bounded(&sm.bar, parity ^ 1u);  // give the copies one more chance to land
-    }
-    __syncthreads();
-    if (sm.abort_flag) return;
-
-    const unsigned char* st = sm.stage;
-    // ---- scores
-    {
-      const int k = tid % G;
-      // warp-uniform trip count: every lane of a warp runs every iteration,
-      // because the group reduction below shuffles across the full warp
-      for (int tb = (tid / 32) * (32 / G); tb < n; tb += kDecThreads / G) {
-        const int t = tb + (tid & 31) / G;
-        const bool valid = t < n;
-        float part[QPG];
-        if (!valid) {
-#pragma unroll
-          for (int hh = 0; hh < QPG; ++hh) part[hh] = 0.f;
-        } else if (s == 0) {
-          const uint4* src = reinterpret_cast<const uint4*>(st + sm.info[4] + t * (2 * D) + k * 64);
-          float x[32];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 u = src[v];
-            const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = half2_bits_to_float2(wds[i]);
-              x[8 * v + 2 * i] = f.x;
-              x[8 * v + 2 * i + 1] = f.y;
-            }
-          }
-#pragma unroll
-          for (int hh = 0; hh < QPG; ++hh) {
-            float dot = 0.f;
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 qq = *reinterpret_cast<const float4*>(&sm.q[hh][k][4 * j4]);
-              dot = fmaf(qq.x, x[4 * j4], dot);
-              dot = fmaf(qq.y, x[4 * j4 + 1], dot);
-              dot = fmaf(qq.z, x[4 * j4 + 2], dot);
-              dot = fmaf(qq.w, x[4 * j4 + 3], dot);
-            }
-            part[hh] = dot;
-          }
-        } else {
-          const uint32_t sp =
-              *reinterpret_cast<const uint32_t*>(st + sm.info[5] + t * (D / kGroup * 4) + k * 4);
-          const float2 sm2 = half2_bits_to_float2(sp);  // (scale, min)
-          float x[32];
-          if (s == 1) {
-            const uint4 u = *reinterpret_cast<const uint4*>(st + sm.info[4] + t * (D / 2) + k * 16);
-            const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd)
-#pragma unroll
-              for (int i = 0; i < 8; ++i) x[8 * wd + i] = code_to_float((wds[wd] >> (4 * i)) & 0xFu);
-          } else {
-            const uint2 u = *reinterpret_cast<const uint2*>(st + sm.info[4] + t * (D / 4) + k * 8);
-            const uint32_t wds[2] = {u.x, u.y};
-#pragma unroll
-            for (int wd = 0; wd < 2; ++wd)
-#pragma unroll
-              for (int i = 0; i < 16; ++i) x[16 * wd + i] = code_to_float((wds[wd] >> (2 * i)) & 0x3u);
-          }
-#pragma unroll
-          for (int hh = 0; hh < QPG; ++hh) {
-            float dot = 0.f;
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 qq = *reinterpret_cast<const float4*>(&sm.q[hh][k][4 * j4]);
-              dot = fmaf(qq.x, x[4 * j4], dot);
-              dot = fmaf(qq.y, x[4 * j4 + 1], dot);
-              dot = fmaf(qq.z, x[4 * j4 + 2], dot);
-              dot = fmaf(qq.w, x[4 * j4 + 3], dot);
-            }
-            part[hh] = fmaf(sm2.x, dot, sm2.y * sm.qsum[hh][k]);
-          }
-        }
-#pragma unroll
-        for (int hh = 0; hh < QPG; ++hh) {
-#pragma unroll
-          for (int off = 1; off < G; off <<= 1) part[hh] += __shfl_xor_sync(0xffffffffu, part[hh], off);
-          if (k == 0 && valid) sm.sc[hh * n + t] = part[hh] * scale_log2;
-        }
-      }
-    }
-    __syncthreads();
-    // ---- softmax statistics per head (log2 domain)
-    {
-      const int warp = tid / 32, lane = tid & 31;
-      for (int hh = warp; hh < QPG; hh += kDecThreads / 32) {
-        float mx = -INFINITY;
-        for (int t = lane; t < n; t += 32) mx = fmaxf(mx, sm.sc[hh * n + t]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        float sum = 0.f;
-        for (int t = lane; t < n; t += 32) {
-          const float p = exp2f(sm.sc[hh * n + t] - mx);
-          sm.sc[hh * n + t] = p;
-          sum += p;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0) {
-          sm.m[hh] = mx;
-          sm.l[hh] = sum;
-        }
-      }
-    }
-    __syncthreads();
-    // ---- values
-    float acc[QPG][8];
-    {
-      const int slice = tid % S, tl = tid / S;
-      const int k = slice / 4;
-      float bias[QPG];
-#pragma unroll
-      for (int hh = 0; hh < QPG; ++hh) {
-        bias[hh] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[hh][i] = 0.f;
-      }
-      for (int t = tl; t < n; t += TL) {
-        float x[8];
-        if (s == 0) {
-          const uint4 u = *reinterpret_cast<const uint4*>(st + sm.info[6] + t * (2 * D) + slice * 16);
-          const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = half2_bits_to_float2(wds[i]);
-            x[2 * i] = f.x;
-            x[2 * i + 1] = f.y;
-          }
-#pragma unroll
-          for (int hh = 0; hh < QPG; ++hh) {
-            const float p = sm.sc[hh * n + t];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[hh][i] = fmaf(p, x[i], acc[hh][i]);
-          }
-        } else {
-          const uint32_t sp =
-              *reinterpret_cast<const uint32_t*>(st + sm.info[7] + t * (D / kGroup * 4) + k * 4);
-          const float2 sm2 = half2_bits_to_float2(sp);
-          if (s == 1) {
-            const uint32_t wd = *reinterpret_cast<const uint32_t*>(st + sm.info[6] + t * (D / 2) + slice * 4);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = code_to_float((wd >> (4 * i)) & 0xFu);
-          } else {
-            const uint32_t wd = *reinterpret_cast<const unsigned short*>(st + sm.info[6] + t * (D / 4) + slice * 2);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = code_to_float((wd >> (2 * i)) & 0x3u);
-          }
-#pragma unroll
-          for (int hh = 0; hh < QPG; ++hh) {
-            const float p = sm.sc[hh * n + t];
-            const float ws = p * sm2.x;
-            bias[hh] = fmaf(p, sm2.y, bias[hh]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[hh][i] = fmaf(ws, x[i], acc[hh][i]);
-          }
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < QPG; ++hh)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[hh][i] += bias[hh];
-    }
-    __syncthreads();  // stage no longer needed: reuse it for the token-lane reduction
-    {
-      float* red = reinterpret_cast<float*>(sm.stage);  // [TL][QPG][D]
-      const int slice = tid % S, tl = tid / S;
-#pragma unroll
-      for (int hh = 0; hh < QPG; ++hh) {
-        float4* dst = reinterpret_cast<float4*>(red + ((size_t)tl * QPG + hh) * D + slice * 8);
-        dst[0] = make_float4(acc[hh][0], acc[hh][1], acc[hh][2], acc[hh][3]);
-        dst[1] = make_float4(acc[hh][4], acc[hh][5], acc[hh][6], acc[hh][7]);
-      }
-    }
-    __syncthreads();
-    {
-      const float* red = reinterpret_cast<const float*>(sm.stage);
-      float* dst = ws_acc + (size_t)w * QPG * D;
-      for (int o = tid; o < QPG * D; o += kDecThreads) {
-        float v = 0.f;
-#pragma unroll
-        for (int tl = 0; tl < TL; ++tl) v += red[(size_t)tl * QPG * D + o];
-        dst[o] = v;
-      }
-      if (tid < QPG) ws_ml[(size_t)w * QPG + tid] = make_float2(sm.m[tid], sm.l[tid]);
-    }
-    __syncthreads();  // stage and scores are rewritten by the next item
+    const unsigned char* regk = packed + r->seg_base[s] + (uint64_t)g * r->region_bytes[s];
+    const unsigned char* regv = regk + (uint64_t)Hkv * r->region_bytes[s];
+    const int64_t qbase = ((int64_t)b * Hkv + g) * QPG * D;
+    if (s == 0)
+      run_item<D, QPG, QDT, 0>(regk, regv, 0, t0, n, q, qbase, scale_log2, ring, w, ws_acc, ws_ml);
+    else if (s == 1)
+      run_item<D, QPG, QDT, 1>(regk, regv, r->scale_offset[1], t0, n, q, qbase, scale_log2, ring, w,
+                               ws_acc, ws_ml);
+    else
+      run_item<D, QPG, QDT, 2>(regk, regv, r->scale_offset[2], t0, n, q, qbase, scale_log2, ring, w,
+                               ws_acc, ws_ml);
   }
 }
 
+// One CTA per (sequence, query head): 8 warps split the items, each keeps a
+// running (max, sum, accumulator) over its items, then the warps' states are
+// merged in shared memory.
 template <int D, int QPG>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
 decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
                       const float* __restrict__ ws_acc, const float2* __restrict__ ws_ml,
                       float* __restrict__ out) {
   constexpr int PER_LANE = D / 32;
+  constexpr int NW = 8;
+  __shared__ float s_acc[NW][D];
+  __shared__ float s_m[NW], s_l[NW];
   const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
-  const int B = h->num_seqs, Hkv = h->num_kv_heads;
-  const int64_t wg = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (wg >= (int64_t)B * Hq) return;
-  const int b = (int)(wg / Hq), hq = (int)(wg % Hq);
+  const int Hkv = h->num_kv_heads;
+  const int64_t bh = blockIdx.x;
+  const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
   const int g = hq / QPG, hh = hq % QPG;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x / 32;
   const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
-  float* o = out + wg * D + lane * PER_LANE;
   const int i0 = r->item_begin[0];
   const int i1 = r->item_begin[2] + r->item_count[2];
-  if (r->num_tokens == 0 || i1 <= i0) {
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) o[i] = 0.f;
-    return;
-  }
-  float M = -INFINITY;
-  for (int it = i0 + lane; it < i1; it += 32) M = fmaxf(M, ws_ml[((int64_t)it * Hkv + g) * QPG + hh].x);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float acc[PER_LANE];
+  float M = -INFINITY, l = 0.f, acc[PER_LANE];
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) acc[i] = 0.f;
-  float l = 0.f;
-  for (int it = i0; it < i1; ++it) {
+  for (int it = i0 + warp; it < i1; it += NW) {
     const int64_t wi = ((int64_t)it * Hkv + g) * QPG + hh;
     const float2 ml = ws_ml[wi];
-    const float f = exp2f(ml.x - M);
-    l = fmaf(f, ml.y, l);
     const float* a = ws_acc + wi * D + lane * PER_LANE;
+    float v[PER_LANE];
     if constexpr (PER_LANE == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(a);
-      acc[0] = fmaf(f, v.x, acc[0]); acc[1] = fmaf(f, v.y, acc[1]);
-      acc[2] = fmaf(f, v.z, acc[2]); acc[3] = fmaf(f, v.w, acc[3]);
+      const float4 t = *reinterpret_cast<const float4*>(a);
+      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
     } else {
-      const float2 v = *reinterpret_cast<const float2*>(a);
-      acc[0] = fmaf(f, v.x, acc[0]); acc[1] = fmaf(f, v.y, acc[1]);
+      const float2 t = *reinterpret_cast<const float2*>(a);
+      v[0] = t.x; v[1] = t.y;
     }
-  }
-  const float inv_l = 1.0f / l;
+    const float Mn = fmaxf(M, ml.x);
+    const float fa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    const float fb = ml.x == -INFINITY ? 0.f : exp2f(ml.x - Mn);
+    l = l * fa + ml.y * fb;
 #pragma unroll
-  for (int i = 0; i < PER_LANE; ++i) o[i] = acc[i] * inv_l;
+    for (int i = 0; i < PER_LANE; ++i) acc[i] = acc[i] * fa + v[i] * fb;
+    M = Mn;
+  }
+#pragma unroll
+  for (int i = 0; i < PER_LANE; ++i) s_acc[warp][lane * PER_LANE + i] = acc[i];
+  if (lane == 0) {
+    s_m[warp] = M;
+    s_l[warp] = l;
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, s_m[w]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float f = s_m[w] == -INFINITY ? 0.f : exp2f(s_m[w] - Mx);
+      num += f * s_acc[w][threadIdx.x];
+      den += f * s_l[w];
+    }
+    out[bh * D + threadIdx.x] = den > 0.f ? num / den : 0.f;
+  }
 }
 
 template <int D, int QPG, int QDT>
@@ -475,7 +565,7 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
                             const unsigned char* packed, const void* q, float scale_log2,
                             float* out, float* ws_acc, float2* ws_ml, int num_seqs,
                             unsigned int* status, cudaStream_t stream) {
-  const size_t smem = sizeof(DecodeSmem);
+  constexpr size_t smem = decode_smem_bytes<D, QPG>();
   auto kern = decode_partial_kernel<D, QPG, QDT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -486,15 +576,15 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
     return err;
   const int64_t cap = max_items;  // work items x kv-heads the workspace holds
   int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
-  if (grid > cap) grid = cap;
+  const int64_t need = (cap + kDecWarps - 1) / kDecWarps;
+  if (grid > need) grid = need;
   if (grid > 0) {
     kern<<<(unsigned)grid, kDecThreads, smem, stream>>>(layout, packed, q, scale_log2, ws_acc, ws_ml,
                                                          cap, status);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const int64_t warps = (int64_t)num_seqs * Hq;
-  decode_combine_kernel<D, QPG><<<(unsigned)((warps + 3) / 4), 128, 0, stream>>>(layout, Hq, ws_acc,
-                                                                                ws_ml, out);
+  const int64_t heads = (int64_t)num_seqs * Hq;
+  decode_combine_kernel<D, QPG><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc, ws_ml, out);
   return cudaGetLastError();
 }
 
