@@ -115,6 +115,31 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ ranks
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own batch: independent problems, no exchange."""
+    return seed + 1009 * rank
+
+
+def reduce_timing(ms_local: float, device=None) -> float:
+    """Max over ranks of the locally measured time (the job ends when the
+    slowest rank ends).  A single process returns its own time."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return ms_local
+    t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ our path
 
 class Setup:
@@ -140,6 +165,9 @@ class Setup:
             self.V.append(V)
             self.q.append([W.query(w, layer, s, seed, device) for s in range(w.decode_steps)])
         u8 = torch.uint8
+        self.route_ws = torch.empty(M.mq_route_workspace_bytes(self.shape, self.lens, w.router_dim,
+                                                                w.router_hidden),
+                                    dtype=u8, device=device)
         self.token_expert = torch.empty(self.T, dtype=u8, device=device)
         self.chunk_expert = torch.empty(max(self.N, 16), dtype=u8, device=device)
         self.layout = torch.empty(M.mq_layout_bytes(self.shape, self.lens), dtype=u8,
@@ -160,7 +188,7 @@ class Setup:
         from chunk_adaptive_mixed_b200 import mqkv as M
         w = self.w
         M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, self.W1, self.W2, self.W3,
-                          self.b3, self.token_expert, self.chunk_expert)
+                          self.b3, self.token_expert, self.chunk_expert, self.route_ws)
         M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_expert, self.layout)
         for layer in range(w.layers):
             if timers:
@@ -179,9 +207,9 @@ class Setup:
                     timers["decode"][layer][1].record()
 
     def launches_per_step(self):
-        # router + vote, 2 layout kernels, one pack per layer, two decode
-        # kernels per layer and decode step
-        return 2 + 2 + self.w.layers + 2 * self.w.layers * self.w.decode_steps
+        # weight split + router + vote, 2 layout kernels, one pack per layer,
+        # two decode kernels per layer and decode step
+        return 3 + 2 + self.w.layers + 2 * self.w.layers * self.w.decode_steps
 
 
 def run_ours(args, rank, world, local_rank):
@@ -194,7 +222,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     w = W.get(args.workload)
-    seed = args.seed + 1009 * rank
+    seed = rank_seed(args.seed, rank)
     S = Setup(w, seed, device)
     dist = world > 1
     if dist:
@@ -230,11 +258,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clocks = sampler.stop()
     assert M.mq_device_status() == 0, "device-side check failed in the timed region"
-    ms = t_start.elapsed_time(t_end)
-    if dist:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_timing(t_start.elapsed_time(t_end), device)
     ms_step = ms / args.steps
     pack_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["pack"]]
     dec_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["decode"]]
@@ -242,7 +266,7 @@ def run_ours(args, rank, world, local_rank):
     dec_avg = float(np.mean(dec_ms))
 
     tokens_per_step = S.B * w.decode_steps
-    value = tokens_per_step * world / (ms_step / 1e3)
+    value = job_throughput(tokens_per_step, world, ms_step)
     peak, peak_kind = measured_peaks()
     pack_bytes = S.kv_bytes + pb                                   # read K/V, write packed
     dec_bytes = pb + sum(x.numel() * x.element_size() for x in (S.q[0][0], S.out[0]))

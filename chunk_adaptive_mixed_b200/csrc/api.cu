@@ -234,11 +234,22 @@ mq_status mq_device_status(uint32_t* h_flags, int32_t clear, void* stream) {
   return MQ_OK;
 }
 
+size_t mq_route_workspace_bytes(const mq_shape* shape, const int32_t* h_seq_lens, int32_t D,
+                                int32_t H) {
+  int64_t T, N;
+  if (check_shape(shape) != MQ_OK || check_lens(shape, h_seq_lens, &T, &N) != MQ_OK) return 0;
+  if (D < 1 || D % 4 != 0 || (H != 64 && H != 128 && H != 256)) {
+    fail(MQ_ERR_INVALID_ARG, "D must be a positive multiple of 4 and H one of 64, 128, 256");
+    return 0;
+  }
+  return route_workspace_bytes(T, D, H);
+}
+
 mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
                           const int64_t* d_cu_seqlens, const float* C, int32_t D, int32_t H,
                           const float* W1, const float* W2, const float* W3, const float* b3,
                           int32_t routing_freeze, uint8_t* token_expert, uint8_t* chunk_expert,
-                          float* logits, void* stream) {
+                          float* logits, void* workspace, size_t workspace_bytes, void* stream) {
   MQ_TRY(check_shape(shape));
   int64_t T, N;
   MQ_TRY(check_lens(shape, h_seq_lens, &T, &N));
@@ -254,16 +265,20 @@ mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
   MQ_NEED_PTR(token_expert, "token_expert");
   MQ_NEED_PTR(chunk_expert, "chunk_expert");
   if (logits && misaligned(logits)) return fail(MQ_ERR_INVALID_ARG, "logits is not 16-byte aligned");
+  const size_t need = route_workspace_bytes(T, D, H);
+  if (workspace_bytes < need)
+    return fail(MQ_ERR_WORKSPACE, "workspace_bytes %zu < %zu needed", workspace_bytes, need);
+  MQ_NEED_PTR(workspace, "workspace");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned int* status = nullptr;
   cudaError_t err = status_word(&status);
   if (err != cudaSuccess) return cuda_fail(err, "device status word");
-  if (T > 0) {
-    err = launch_router(C, T, D, H, W1, W2, W3, b3, token_expert, logits, st);
-    if (err != cudaSuccess) return cuda_fail(err, "router launch");
-  }
-  err = launch_vote(shape->num_seqs, d_cu_seqlens, shape->chunk_len, token_expert, routing_freeze,
-                    chunk_expert, status, st);
+  const float4* zpart = nullptr;
+  int nhb = 0;
+  err = launch_router_tc(C, T, D, H, W1, W2, W3, workspace, status, st, &zpart, &nhb);
+  if (err != cudaSuccess) return cuda_fail(err, "router launch");
+  err = launch_finish_vote(shape->num_seqs, d_cu_seqlens, shape->chunk_len, zpart, nhb, b3,
+                           routing_freeze, token_expert, logits, chunk_expert, st);
   if (err != cudaSuccess) return cuda_fail(err, "vote launch");
   return MQ_OK;
 }

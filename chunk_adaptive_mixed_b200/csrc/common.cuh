@@ -102,12 +102,18 @@ struct ItemPolicy {
 ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens);
 int64_t max_items_per_kv_head(const mq_shape& s, const int32_t* h_seq_lens, const ItemPolicy& p);
 
-cudaError_t launch_router(const float* C, int64_t T, int D, int H, const float* W1,
-                          const float* W2, const float* W3, const float* b3,
-                          uint8_t* token_expert, float* logits, cudaStream_t stream);
-cudaError_t launch_vote(int B, const int64_t* cu_seqlens, int L, const uint8_t* token_expert,
-                        int routing_freeze, uint8_t* chunk_expert, unsigned int* status,
-                        cudaStream_t stream);
+// Router on tcgen05 (3 x TF32): weights pre-split into the workspace, then
+// per-hidden-block partial scores; finish_vote sums them, adds the bias, takes
+// the argmax and the chunk vote.
+size_t route_workspace_bytes(int64_t T, int D, int H);
+cudaError_t launch_router_tc(const float* C, int64_t T, int D, int H, const float* W1,
+                             const float* W2, const float* W3, void* workspace,
+                             unsigned int* status, cudaStream_t stream, const float4** zpart_out,
+                             int* nhb_out);
+cudaError_t launch_finish_vote(int B, const int64_t* cu_seqlens, int L, const float4* zpart,
+                               int nhb, const float* b3, int routing_freeze,
+                               uint8_t* token_expert, float* logits, uint8_t* chunk_expert,
+                               cudaStream_t stream);
 cudaError_t launch_layout(const mq_shape& s, const int64_t* cu_seqlens, const uint8_t* chunk_expert,
                           int64_t total_chunks, const ItemPolicy& pol, void* layout,
                           unsigned int* status, cudaStream_t stream);

@@ -35,7 +35,7 @@ MQ_DEV_INDEX_RANGE = 0x10
 
 # names of every function include/mqkv.h declares
 EXPORTS = ("mq_status_string", "mq_last_error", "mq_layout_bytes", "mq_packed_bytes_upper_bound",
-           "mq_decode_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
+           "mq_decode_workspace_bytes", "mq_route_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
            "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc")
 
 # size of the scratch array built into the library for mq_decode_attn_noalloc
@@ -84,8 +84,11 @@ def lib() -> ctypes.CDLL:
     L.mq_packed_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t), vp]
     L.mq_device_status.restype = ctypes.c_int
     L.mq_device_status.argtypes = [u32p, i32, vp]
+    L.mq_route_workspace_bytes.restype = sz
+    L.mq_route_workspace_bytes.argtypes = [sp, vp, i32, i32]
     L.mq_route_chunks.restype = ctypes.c_int
-    L.mq_route_chunks.argtypes = [sp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+    L.mq_route_chunks.argtypes = [sp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp,
+                                  sz, vp]
     L.mq_build_layout.restype = ctypes.c_int
     L.mq_build_layout.argtypes = [sp, vp, vp, vp, vp, sz, vp]
     L.mq_pack_kv.restype = ctypes.c_int
@@ -186,14 +189,23 @@ def mq_device_status(clear: bool = True, stream=None) -> int:
 
 # ---------------------------------------------------------------- the path
 
+def mq_route_workspace_bytes(shp, seq_lens, D, H) -> int:
+    l = _lens(seq_lens)
+    n = lib().mq_route_workspace_bytes(ctypes.byref(shp), l.ctypes.data, int(D), int(H))
+    if n == 0:
+        raise MqkvError(MQ_ERR_INVALID_ARG, last_error())
+    return int(n)
+
+
 def mq_route_chunks(shp, seq_lens, cu_seqlens, C, W1, W2, W3, b3, token_expert, chunk_expert,
-                    logits=None, routing_freeze=True, stream=None):
+                    workspace, logits=None, routing_freeze=True, stream=None):
     l = _lens(seq_lens)
     D, H = int(C.shape[1]), int(W1.shape[1])
+    nbytes = workspace.numel() * workspace.element_size()
     _check(lib().mq_route_chunks(ctypes.byref(shp), l.ctypes.data, _ptr(cu_seqlens), _ptr(C), D, H,
                                  _ptr(W1), _ptr(W2), _ptr(W3), _ptr(b3), int(bool(routing_freeze)),
                                  _ptr(token_expert), _ptr(chunk_expert), _ptr(logits),
-                                 _stream(stream)), "mq_route_chunks")
+                                 _ptr(workspace), nbytes, _stream(stream)), "mq_route_chunks")
 
 
 def mq_build_layout(shp, seq_lens, cu_seqlens, chunk_expert, layout, stream=None):

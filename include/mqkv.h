@@ -240,15 +240,25 @@ mq_status mq_device_status(uint32_t* h_flags, int32_t clear, void* stream);
  *   chunk_expert device uint8 [N]  out: per-chunk expert, chunk (b, c) at
  *                                  index chunk_offset_b + c
  *   logits       device fp32 [T, 3] out, or NULL
+ *   workspace    device buffer of at least mq_route_workspace_bytes(shape,
+ *                h_seq_lens, D, H) bytes (weights split for the tensor
+ *                cores, partial scores); contents on entry are ignored
  * Constraints: 1 <= D, D % 4 == 0; H in {64, 128, 256}.
+ * The two projections run on the tensor cores in three tf32 passes
+ * (hi*hi + hi*lo + lo*hi of a tf32 high part and an fp32 remainder), which
+ * keeps each product within about 2^-21 relative of fp32.
  * ------------------------------------------------------------------------- */
+size_t mq_route_workspace_bytes(const mq_shape* shape, const int32_t* h_seq_lens,
+                                int32_t D, int32_t H);
+
 mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
                           const int64_t* d_cu_seqlens,
                           const float* C, int32_t D, int32_t H,
                           const float* W1, const float* W2, const float* W3,
                           const float* b3, int32_t routing_freeze,
                           uint8_t* token_expert, uint8_t* chunk_expert,
-                          float* logits, void* stream);
+                          float* logits, void* workspace, size_t workspace_bytes,
+                          void* stream);
 
 /* ---------------------------------------------------------------------------
  * mq_build_layout — Cocktail's chunk regrouping (chunk-level KV cache

@@ -15,6 +15,12 @@ REL_L2 = 1e-3
 MAX_ABS = 4e-3
 # router scores: tokens whose fp64 top-2 gap is below this may flip
 NEAR_TIE = 1e-3
+# Score error allowed against the fp64 oracle.  A token's argmax can change
+# only if some score moves by half its top-2 gap or more, so any error below
+# NEAR_TIE / 2 keeps every choice outside the near-tie band exact.  The
+# tensor-core accumulator truncates once per MMA (about D/8 * 2^-24 relative),
+# which reaches ~1.5e-4 at D = 5120; 4e-4 keeps a margin under NEAR_TIE / 2.
+SCORE_TOL = 4e-4
 
 
 def dev():
@@ -70,7 +76,9 @@ def gpu_route(case, C, W1, W2, W3, b3, freeze=True):
     te = torch.empty(max(case.T, 16), dtype=torch.uint8, device=dev())
     ce = torch.empty(max(case.N, 16), dtype=torch.uint8, device=dev())
     logits = torch.empty(max(case.T, 1), 3, dtype=torch.float32, device=dev())
-    M.mq_route_chunks(shp, case.lens, case.cu(), C, W1, W2, W3, b3, te, ce, logits,
+    ws = torch.empty(M.mq_route_workspace_bytes(shp, case.lens, C.shape[1], W1.shape[1]),
+                     dtype=torch.uint8, device=dev())
+    M.mq_route_chunks(shp, case.lens, case.cu(), C, W1, W2, W3, b3, te, ce, ws, logits,
                       routing_freeze=freeze)
     torch.cuda.synchronize()
     assert M.mq_device_status() == 0
@@ -163,7 +171,7 @@ def check_route(lens, L, te_gpu, ce_gpu, logits_gpu, z32, z64, freeze=True):
     gap = O.top2_gap(z64)
     near = gap < NEAR_TIE
     scale = np.maximum(1.0, np.abs(z64))
-    assert np.all(np.abs(logits_gpu - z64) <= 1e-4 * scale), \
+    assert np.all(np.abs(logits_gpu - z64) <= SCORE_TOL * scale), \
         f"router scores differ: max {np.abs(logits_gpu - z64).max():.3e}"
     bad = (te_gpu != te_o) & ~near
     assert not bad.any(), f"{bad.sum()} token choices differ away from ties"

@@ -96,9 +96,15 @@ def test_bad_pointers_and_sizes():
         == M.MQ_ERR_INVALID_ARG
     # router: H unsupported, D not a multiple of 4
     assert lib.mq_route_chunks(ctypes.byref(shp), lens.ctypes.data, p, p, 64, 96, p, p, p, None, 1,
-                               p, p, None, 0) == M.MQ_ERR_UNSUPPORTED
+                               p, p, None, p, 1 << 30, 0) == M.MQ_ERR_UNSUPPORTED
     assert lib.mq_route_chunks(ctypes.byref(shp), lens.ctypes.data, p, p, 66, 64, p, p, p, None, 1,
-                               p, p, None, 0) == M.MQ_ERR_INVALID_ARG
+                               p, p, None, p, 1 << 30, 0) == M.MQ_ERR_INVALID_ARG
+    # router workspace too small
+    rws = lib.mq_route_workspace_bytes(ctypes.byref(shp), lens.ctypes.data, 64, 64)
+    assert rws > 0
+    assert lib.mq_route_chunks(ctypes.byref(shp), lens.ctypes.data, p, p, 64, 64, p, p, p, None, 1,
+                               p, p, None, p, rws - 1, 0) == M.MQ_ERR_WORKSPACE
+    assert lib.mq_route_workspace_bytes(ctypes.byref(shp), lens.ctypes.data, 64, 100) == 0
     # layout buffer too small
     need = lib.mq_layout_bytes(ctypes.byref(shp), lens.ctypes.data)
     assert lib.mq_build_layout(ctypes.byref(shp), lens.ctypes.data, p, p, p, need - 16, 0) \
