@@ -32,6 +32,7 @@ namespace {
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kRing = 4;  // stages of each warp's copy ring
+constexpr float kRescale = 8.0f;
 
 // Lane geometry of one precision: each lane owns SL consecutive dims of one
 // token (SL * QPG query values and accumulators stay in registers), LPT lanes
@@ -268,10 +269,16 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
           st + 2 * Gm::CODES + Gm::SCALES + tl * Gm::SROW + grp * 4));
       ks = a.x; km = a.y; vs = b.x; vm = b.y;
     }
-    // ---- scores: q . code (pairs), then the group's scale and min
-    uint64_t dot2[QPG];
+    // ---- scores: q . code (pairs) in kChains independent accumulator chains
+    // (short dependency chains), then the group's scale and min
+    // (with several query heads per kv-head the heads already give independent
+    // chains)
+    constexpr int kChains = QPG > 1 ? 1 : (NP >= 4 ? 4 : NP);
+    uint64_t dot2[QPG][kChains];
 #pragma unroll
-    for (int h = 0; h < QPG; ++h) dot2[h] = 0ull;
+    for (int h = 0; h < QPG; ++h)
+#pragma unroll
+      for (int c = 0; c < kChains; ++c) dot2[h][c] = 0ull;
     if constexpr (E == 0) {
       const uint32_t* wv = reinterpret_cast<const uint32_t*>(kp);
 #pragma unroll
@@ -279,7 +286,7 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
         const float2 f = half2_bits_to_float2(wv[i]);
         const uint64_t x = pk2(f.x, f.y);
 #pragma unroll
-        for (int h = 0; h < QPG; ++h) dot2[h] = fma2(x, qp[h][i], dot2[h]);
+        for (int h = 0; h < QPG; ++h) dot2[h][i % kChains] = fma2(x, qp[h][i], dot2[h][i % kChains]);
       }
     } else {
       constexpr int BYTES = SL * BITS / 8;
@@ -296,14 +303,16 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
         if constexpr (BITS == 4) {
           const uint64_t x = pk2u(t & 0xFF0F0000u, t & 0xFF00F000u);
 #pragma unroll
-          for (int h = 0; h < QPG; ++h) dot2[h] = fma2(x, qp[h][mb], dot2[h]);
+          for (int h = 0; h < QPG; ++h)
+            dot2[h][mb % kChains] = fma2(x, qp[h][mb], dot2[h][mb % kChains]);
         } else {
           const uint64_t x0 = pk2u(t & 0xFF030000u, t & 0xFF0C0000u);
           const uint64_t x1 = pk2u(t & 0xFF300000u, t & 0xFF00C000u);
 #pragma unroll
           for (int h = 0; h < QPG; ++h) {
-            dot2[h] = fma2(x0, qp[h][2 * mb], dot2[h]);
-            dot2[h] = fma2(x1, qp[h][2 * mb + 1], dot2[h]);
+            dot2[h][(2 * mb) % kChains] = fma2(x0, qp[h][2 * mb], dot2[h][(2 * mb) % kChains]);
+            dot2[h][(2 * mb + 1) % kChains] =
+                fma2(x1, qp[h][2 * mb + 1], dot2[h][(2 * mb + 1) % kChains]);
           }
         }
       }
@@ -311,7 +320,9 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
     float part[QPG];
 #pragma unroll
     for (int h = 0; h < QPG; ++h) {
-      const float dot = lo2(dot2[h]) + hi2(dot2[h]);
+      float dot = 0.f;
+#pragma unroll
+      for (int c = 0; c < kChains; ++c) dot += lo2(dot2[h][c]) + hi2(dot2[h][c]);
       part[h] = E == 0 ? dot : fmaf(ks, dot - qb[h], km * qs[h]);
     }
 #pragma unroll
@@ -322,7 +333,10 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
 #pragma unroll
     for (int h = 0; h < QPG; ++h) {
       const float sc = valid ? part[h] * scale_log2 : -INFINITY;
-      if (sc > m[h]) {  // new running maximum: rescale what was accumulated
+      // lazy rescaling: the reference maximum moves only when a score exceeds
+      // it by more than kRescale (log2 units), so weights stay below
+      // 2^kRescale; (m, l, acc) remain consistent for any reference
+      if (sc > m[h] + kRescale) {
         const float a = exp2f(m[h] - sc);
         const uint64_t a2 = pk2(a, a);
         l[h] *= a;
