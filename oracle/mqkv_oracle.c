@@ -208,6 +208,51 @@ void mqo_route(int B, const int32_t* seq_lens, int L, int D, int H, const float*
   mqo_vote(B, seq_lens, L, token_expert, routing_freeze, chunk_expert);
 }
 
+/* -------------------------------------------------- similarity search */
+
+/*
+ * Chunk-level quantization search by similarity (Cocktail abstract on the
+ * "Bin Zhang" scholarfeed author page: the bitwidth of each context chunk is
+ * chosen from the similarity between the chunk and the query).  The page
+ * gives neither the similarity nor the thresholds; the reading used here:
+ *   sim(b, c) = cos(mean of C_t over the chunk's tokens, u_b)   (fp64)
+ *   expert = FP16 if sim >= tau_hi, INT4 if sim >= tau_lo, else INT2;
+ *   a zero vector gives sim = 0; with routing_freeze, chunk 0 is FP16.
+ * C [T, D] fp32 (sequences back to back), u [B, D] fp32.
+ */
+void mqo_similarity_route(int B, const int32_t* seq_lens, int L, int D, const float* C,
+                          const float* u, double tau_hi, double tau_lo, int routing_freeze,
+                          uint8_t* chunk_expert, double* sim_out) {
+  int64_t row = 0, ci = 0;
+  double* mean = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int b = 0; b < B; ++b) {
+    const int Tb = seq_lens[b];
+    const int nb = (Tb + L - 1) / L;
+    double unorm = 0.0;
+    for (int k = 0; k < D; ++k) unorm += (double)u[(int64_t)b * D + k] * u[(int64_t)b * D + k];
+    for (int c = 0; c < nb; ++c) {
+      const int t0 = c * L, t1 = (t0 + L < Tb) ? t0 + L : Tb;
+      for (int k = 0; k < D; ++k) mean[k] = 0.0;
+      for (int t = t0; t < t1; ++t)
+        for (int k = 0; k < D; ++k) mean[k] += (double)C[(row + t) * (int64_t)D + k];
+      double dot = 0.0, mnorm = 0.0;
+      for (int k = 0; k < D; ++k) {
+        mean[k] /= (double)(t1 - t0);
+        dot += mean[k] * (double)u[(int64_t)b * D + k];
+        mnorm += mean[k] * mean[k];
+      }
+      const double sim = (mnorm > 0.0 && unorm > 0.0) ? dot / sqrt(mnorm * unorm) : 0.0;
+      int e = sim >= tau_hi ? 0 : (sim >= tau_lo ? 1 : 2);
+      if (routing_freeze && c == 0) e = 0;
+      chunk_expert[ci + c] = (uint8_t)e;
+      if (sim_out) sim_out[ci + c] = sim;
+    }
+    row += Tb;
+    ci += nb;
+  }
+  free(mean);
+}
+
 /* --------------------------------------------------------------- layout */
 
 /* Layout table as the public header describes it, rebuilt here from prose. */

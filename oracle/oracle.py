@@ -64,6 +64,9 @@ def lib():
         L.mqo_dense_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           _i32p, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int,
                                           ctypes.c_double, _f64p]
+        L.mqo_similarity_route.argtypes = [ctypes.c_int, _i32p, ctypes.c_int, ctypes.c_int, _f32p,
+                                           _f32p, ctypes.c_double, ctypes.c_double, ctypes.c_int,
+                                           _u8p, _f64p]
         L.mqo_f32_to_f16.argtypes = [_f32p, _u16p, ctypes.c_int64]
         L.mqo_f16_to_f32.argtypes = [_u16p, _f32p, ctypes.c_int64]
         _LIB = L
@@ -157,6 +160,22 @@ def route(seq_lens, L, C, W1, W2, W3, b3=None, routing_freeze=True):
                     int(bool(routing_freeze)), _p(te, _u8p), _p(ce, _u8p), _p(z32, _f32p),
                     _p(z64, _f64p))
     return ce, te, z32, z64
+
+
+def similarity_route(seq_lens, L, C, u, tau_hi, tau_lo, routing_freeze=True):
+    """Returns (chunk_expert, fp64 similarity per chunk)."""
+    sl = _c(seq_lens, np.int32)
+    C = _c(C, np.float32)
+    u = _c(u, np.float32)
+    D = C.shape[1]
+    assert u.shape == (len(sl), D) and C.shape[0] == int(sl.sum())
+    n = num_chunks(sl, L)
+    ce = np.empty(n, np.uint8)
+    sim = np.empty(n, np.float64)
+    lib().mqo_similarity_route(len(sl), _p(sl, _i32p), int(L), D, _p(C, _f32p), _p(u, _f32p),
+                               float(tau_hi), float(tau_lo), int(bool(routing_freeze)),
+                               _p(ce, _u8p), _p(sim, _f64p))
+    return ce, sim
 
 
 def layout_bytes(seq_lens, L):

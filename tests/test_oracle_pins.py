@@ -533,3 +533,46 @@ def test_decode_pairs_agrees_with_decode():
     pairs = np.array([[b, h] for b in range(2) for h in range(Hq)], np.int32)
     op = O.decode_pairs(Hq, Hkv, d, L, lens, ce, K, V, q, pairs)
     assert np.array_equal(op.reshape(2, Hq, d), o)
+
+
+# ------------------------------------------------------ similarity search
+
+def test_similarity_route_closed_forms():
+    # chunk rows built as exact multiples of u: cos = +1, -1, 0 (orthogonal)
+    D, L = 8, 32
+    u = np.zeros((1, D), np.float32)
+    u[0, :4] = [1.0, 2.0, -1.0, 0.5]
+    ortho = np.zeros(D, np.float32)
+    ortho[4:] = [3.0, -1.0, 2.0, 1.0]                  # disjoint support: orthogonal to u
+    rows = []
+    for c, v in enumerate([u[0] * 2.0, -u[0], ortho, u[0] + 0.0 * ortho]):
+        rows.append(np.tile(v, (L, 1)))
+    C = np.concatenate(rows).astype(np.float32)
+    lens = np.array([4 * L], np.int32)
+    ce, sim = O.similarity_route(lens, L, C, u, tau_hi=0.9, tau_lo=-0.5, routing_freeze=False)
+    assert np.allclose(sim, [1.0, -1.0, 0.0, 1.0], atol=1e-12)
+    assert ce.tolist() == [0, 2, 1, 0]
+    ce, _ = O.similarity_route(lens, L, C, u, tau_hi=0.9, tau_lo=-0.5, routing_freeze=True)
+    assert ce.tolist() == [0, 2, 1, 0]
+    # the similarity uses the chunk MEAN: varying rows whose mean is u give 1
+    noise = np.random.default_rng(0).standard_normal((L, D)).astype(np.float32)
+    noise -= noise.mean(axis=0, keepdims=True)
+    C2 = (np.tile(u[0], (L, 1)) + noise).astype(np.float64)
+    C2 -= C2.mean(axis=0) - u[0]                      # exact mean = u (up to fp32)
+    _, sim2 = O.similarity_route(np.array([L], np.int32), L, C2.astype(np.float32), u, 0.5, 0.0,
+                                 routing_freeze=False)
+    assert abs(sim2[0] - 1.0) < 1e-6
+
+
+def test_similarity_route_tail_zero_and_freeze():
+    D, L = 4, 32
+    u = np.array([[1.0, 0.0, 0.0, 0.0], [0.0, 0.0, 0.0, 0.0]], np.float32)
+    lens = np.array([40, 5], np.int32)                # tail chunk of 8 tokens; second seq u = 0
+    C = np.zeros((45, D), np.float32)
+    C[32:40, 0] = -2.0                                # tail chunk anti-aligned
+    C[40:45, 1] = 1.0
+    ce, sim = O.similarity_route(lens, L, C, u, tau_hi=0.5, tau_lo=0.25, routing_freeze=False)
+    assert sim.tolist() == [0.0, -1.0, 0.0]           # zero mean chunk 0, tail -1, u = 0
+    assert ce.tolist() == [2, 2, 2]
+    ce, _ = O.similarity_route(lens, L, C, u, tau_hi=0.5, tau_lo=0.25, routing_freeze=True)
+    assert ce.tolist() == [0, 2, 0]
