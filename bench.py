@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-rs", action="store_true",
+                   help="routing sharing off: one router, map and layout per layer")
     return p.parse_args()
 
 
@@ -145,7 +147,7 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
 class Setup:
     """Device-resident inputs and outputs of one batch of the workload."""
 
-    def __init__(self, w, seed, device):
+    def __init__(self, w, seed, device, routing_sharing=True):
         import torch
         from chunk_adaptive_mixed_b200 import mqkv as M
         from chunk_adaptive_mixed_b200 import workloads as W
@@ -156,7 +158,14 @@ class Setup:
         self.N = int(W.num_chunks(self.lens, w.chunk_len).sum())
         self.shape = M.shape(self.B, w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_len)
         self.cu = torch.as_tensor(W.cu_seqlens(self.lens), device=device)
-        self.W1, self.W2, self.W3, self.b3 = W.router_weights(w, seed, device)
+        self.rs = routing_sharing
+        # with routing sharing one router serves every layer; without it each
+        # layer has its own router (weights drawn from seed + layer) over the
+        # same router input, so each layer gets its own map and layout
+        nr = 1 if routing_sharing else w.layers
+        self.routers = [W.router_weights(w, seed + (l if not routing_sharing else 0), device)
+                        for l in range(nr)]
+        self.W1, self.W2, self.W3, self.b3 = self.routers[0]
         self.C = W.router_input(w, self.lens, seed, device)
         self.K, self.V, self.q = [], [], []
         for layer in range(w.layers):
@@ -169,9 +178,12 @@ class Setup:
                                                                 w.router_hidden),
                                     dtype=u8, device=device)
         self.token_expert = torch.empty(self.T, dtype=u8, device=device)
-        self.chunk_expert = torch.empty(max(self.N, 16), dtype=u8, device=device)
-        self.layout = torch.empty(M.mq_layout_bytes(self.shape, self.lens), dtype=u8,
-                                  device=device)
+        self.chunk_experts = [torch.empty(max(self.N, 16), dtype=u8, device=device)
+                              for _ in range(nr)]
+        self.layouts = [torch.empty(M.mq_layout_bytes(self.shape, self.lens), dtype=u8,
+                                    device=device) for _ in range(nr)]
+        self.chunk_expert = self.chunk_experts[0]
+        self.layout = self.layouts[0]
         # packed buffers sized for any routing map (all-FP16 bound): no host
         # round trip is needed between routing and packing
         ub = M.mq_packed_bytes_upper_bound(self.shape, self.lens)
@@ -187,29 +199,34 @@ class Setup:
         """One pass of the whole path (launches only; asynchronous)."""
         from chunk_adaptive_mixed_b200 import mqkv as M
         w = self.w
-        M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, self.W1, self.W2, self.W3,
-                          self.b3, self.token_expert, self.chunk_expert, self.route_ws)
-        M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_expert, self.layout)
+        for r, (W1, W2, W3, b3) in enumerate(self.routers):
+            M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, W1, W2, W3, b3,
+                              self.token_expert, self.chunk_experts[r], self.route_ws)
+            M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_experts[r],
+                              self.layouts[r])
         for layer in range(w.layers):
             if timers:
                 timers["pack"][layer][0].record()
-            M.mq_pack_kv(self.shape, self.lens, self.layout, self.K[layer], self.V[layer],
-                         self.packed[layer])
+            M.mq_pack_kv(self.shape, self.lens, self.layout_of(layer), self.K[layer],
+                         self.V[layer], self.packed[layer])
             if timers:
                 timers["pack"][layer][1].record()
         for s in range(w.decode_steps):
             for layer in range(w.layers):
                 if timers and s == 0:
                     timers["decode"][layer][0].record()
-                M.mq_decode_attn(self.shape, self.lens, self.layout, self.packed[layer],
-                                 self.q[layer][s], self.out[layer], self.ws)
+                M.mq_decode_attn(self.shape, self.lens, self.layout_of(layer),
+                                 self.packed[layer], self.q[layer][s], self.out[layer], self.ws)
                 if timers and s == 0:
                     timers["decode"][layer][1].record()
 
+    def layout_of(self, layer):
+        return self.layouts[0 if self.rs else layer]
+
     def launches_per_step(self):
-        # weight split + router + vote, 2 layout kernels, one pack per layer,
-        # two decode kernels per layer and decode step
-        return 3 + 2 + self.w.layers + 2 * self.w.layers * self.w.decode_steps
+        # per router: weight split + router + vote and 2 layout kernels; one
+        # pack per layer; two decode kernels per layer and decode step
+        return 5 * len(self.routers) + self.w.layers + 2 * self.w.layers * self.w.decode_steps
 
 
 def run_ours(args, rank, world, local_rank):
@@ -223,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     w = W.get(args.workload)
     seed = rank_seed(args.seed, rank)
-    S = Setup(w, seed, device)
+    S = Setup(w, seed, device, routing_sharing=not args.no_rs)
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -236,7 +253,7 @@ def run_ours(args, rank, world, local_rank):
         S.step()
     torch.cuda.synchronize()
     assert M.mq_device_status() == 0, "device-side check failed during warm-up"
-    pb = M.mq_packed_bytes(S.layout)
+    pb = int(np.mean([M.mq_packed_bytes(S.layout_of(l)) for l in range(w.layers)]))
     mix = np.bincount(S.chunk_expert[:S.N].cpu().numpy(), minlength=3) / max(S.N, 1)
 
     # per-kernel events for every pack launch and the first decode step
@@ -293,6 +310,7 @@ def run_ours(args, rank, world, local_rank):
                        "head_dim": w.head_dim, "chunk_len": w.chunk_len,
                        "router_D": w.router_dim, "router_H": w.router_hidden,
                        "kv_dtype": w.kv_dtype, "decode_steps": w.decode_steps,
+                       "routing_sharing": S.rs,
                        "parallelism": f"dp{world} (independent batches)",
                        "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
                        else "inputs fit in L2"},

@@ -277,7 +277,12 @@ mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
   int nhb = 0;
   err = launch_router_tc(C, T, D, H, W1, W2, W3, workspace, status, st, &zpart, &nhb);
   if (err != cudaSuccess) return cuda_fail(err, "router launch");
-  err = launch_finish_vote(shape->num_seqs, d_cu_seqlens, shape->chunk_len, zpart, nhb, b3,
+  int64_t max_chunks = 0;
+  for (int b = 0; b < shape->num_seqs; ++b) {
+    const int64_t nb = (h_seq_lens[b] + shape->chunk_len - 1) / shape->chunk_len;
+    max_chunks = nb > max_chunks ? nb : max_chunks;
+  }
+  err = launch_finish_vote(shape->num_seqs, d_cu_seqlens, shape->chunk_len, max_chunks, zpart, nhb, b3,
                            routing_freeze, token_expert, logits, chunk_expert, st);
   if (err != cudaSuccess) return cuda_fail(err, "vote launch");
   return MQ_OK;

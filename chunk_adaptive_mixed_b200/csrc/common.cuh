@@ -110,8 +110,8 @@ cudaError_t launch_router_tc(const float* C, int64_t T, int D, int H, const floa
                              const float* W2, const float* W3, void* workspace,
                              unsigned int* status, cudaStream_t stream, const float4** zpart_out,
                              int* nhb_out);
-cudaError_t launch_finish_vote(int B, const int64_t* cu_seqlens, int L, const float4* zpart,
-                               int nhb, const float* b3, int routing_freeze,
+cudaError_t launch_finish_vote(int B, const int64_t* cu_seqlens, int L, int64_t max_chunks,
+                               const float4* zpart, int nhb, const float* b3, int routing_freeze,
                                uint8_t* token_expert, float* logits, uint8_t* chunk_expert,
                                cudaStream_t stream);
 cudaError_t launch_layout(const mq_shape& s, const int64_t* cu_seqlens, const uint8_t* chunk_expert,

@@ -352,7 +352,7 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   }
 }
 
-// One CTA per sequence, one warp per chunk: sum the hidden-block partial
+// CTA (sequence b, block of 8 chunks), one warp per chunk: sum the hidden-block partial
 // scores, add the bias, take each token's argmax (ties -> lower index = more
 // bits), write them, and take the chunk's majority (ties -> more bits);
 // chunk 0 is frozen to FP16 when asked (路由冻结).
@@ -363,18 +363,20 @@ __global__ void finish_vote_kernel(const int64_t* __restrict__ cu, int L,
                                    uint8_t* __restrict__ chunk_expert) {
   __shared__ int64_t red[32];
   const int b = blockIdx.x;
-  const int64_t coff = block_chunk_offset(b, cu, L, red);
   const int64_t row0 = cu[b];
   const int64_t Tb = cu[b + 1] - row0;
   const int64_t nb = (Tb + L - 1) / L;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+  const int nw = blockDim.x / 32;
+  if ((int64_t)blockIdx.y * nw >= nb) return;  // uniform for the whole block
+  const int64_t coff = block_chunk_offset(b, cu, L, red);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x / 32 + blockIdx.y * nw;
   float bias0 = 0.f, bias1 = 0.f, bias2 = 0.f;
   if (b3) {
     bias0 = b3[0];
     bias1 = b3[1];
     bias2 = b3[2];
   }
-  for (int64_t c = warp; c < nb; c += nw) {
+  for (int64_t c = warp; c < nb; c += (int64_t)nw * gridDim.y) {
     const int64_t t0 = c * L;
     const int64_t t1 = min(t0 + (int64_t)L, Tb);
     int cnt[kNumExperts] = {0, 0, 0};
@@ -462,12 +464,13 @@ cudaError_t launch_router_tc(const float* C, int64_t T, int D, int H, const floa
   return launch_tc<128>(C, T, D, H, W1, W2, W3, Wp, zpart, status, stream);
 }
 
-cudaError_t launch_finish_vote(int B, const int64_t* cu_seqlens, int L, const float4* zpart,
-                               int nhb, const float* b3, int routing_freeze,
+cudaError_t launch_finish_vote(int B, const int64_t* cu_seqlens, int L, int64_t max_chunks,
+                               const float4* zpart, int nhb, const float* b3, int routing_freeze,
                                uint8_t* token_expert, float* logits, uint8_t* chunk_expert,
                                cudaStream_t stream) {
-  finish_vote_kernel<<<B, 256, 0, stream>>>(cu_seqlens, L, zpart, nhb, b3, routing_freeze,
-                                            token_expert, logits, chunk_expert);
+  const int64_t chunk_blocks = max_chunks > 0 ? (max_chunks + 7) / 8 : 1;  // 8 warps a block
+  finish_vote_kernel<<<dim3(B, (unsigned)chunk_blocks), 256, 0, stream>>>(
+      cu_seqlens, L, zpart, nhb, b3, routing_freeze, token_expert, logits, chunk_expert);
   return cudaGetLastError();
 }
 

@@ -178,3 +178,39 @@ def test_stream_ordering_on_a_side_stream():
     ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, K.numpy(), V.numpy())
     want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
     check_attention(out, want, "side stream")
+
+
+def test_routing_sharing_off_gives_each_layer_its_own_map_and_layout():
+    """Routing sharing off (MoQAE notes, ablation without RS): every layer has
+    its own router, so its own map, layout and packed cache; each layer is
+    checked against the oracle with its own map."""
+    lens = np.array([700, 300], np.int32)
+    case = Case(lens, 8, 4, 128, 64)
+    D, H = 64, 64
+    g = torch.Generator().manual_seed(77)
+    C = torch.randn(case.T, D, generator=g)
+    maps = []
+    for layer in range(3):
+        W1 = torch.randn(D, H, generator=g) / D ** 0.5
+        W2 = torch.randn(D, H, generator=g) / D ** 0.5
+        W3 = torch.randn(H, 3, generator=g) / H ** 0.5
+        b3 = torch.tensor([0.0, 0.3, 0.1])
+        te, ce, logits = gpu_route(case, C.to(dev()), W1.to(dev()), W2.to(dev()), W3.to(dev()),
+                                   b3.to(dev()))
+        ce_o, _, z32, z64 = O.route(lens, case.L, C.numpy(), W1.numpy(), W2.numpy(), W3.numpy(),
+                                    b3.numpy())
+        _, exempt = check_route(lens, case.L, te, ce, logits, z32, z64)
+        maps.append(ce_o)
+        K, V, q = random_kv(case, seed=100 + layer)
+        layout = gpu_layout(case, ce)                      # the GPU's own map
+        packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+        out = gpu_decode(case, layout, packed, q.to(dev()))
+        ref = O.pack(case.Hkv, case.d, case.L, lens, ce_o, K.numpy(), V.numpy())
+        want = O.decode(case.Hq, case.Hkv, case.d, case.L, lens, ce_o, ref, q.numpy())
+        if np.array_equal(ce, ce_o):
+            check_layout(case, layout.cpu().numpy(), ce_o)
+            assert np.array_equal(packed[:pb].cpu().numpy(), ref)
+            check_attention(out, want, f"layer {layer}")
+        else:
+            assert exempt > 0
+    assert any(not np.array_equal(maps[0], m) for m in maps[1:])
