@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--router", default="moqae", choices=["moqae", "similarity"],
+                   help="chunk map from MoQAE's router or from Cocktail's chunk-query similarity")
     p.add_argument("--no-rs", action="store_true",
                    help="routing sharing off: one router, map and layout per layer")
     return p.parse_args()
@@ -59,6 +61,34 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def peaks_all():
+    """{hbm GB/s, tf32 TFLOP/s}: the measured copy bandwidth, and the measured
+    bf16 GEMM burst rate times the nominal dense tf32/bf16 ratio (1.1 / 2.25)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm": float(d["hbm_gbs"]), "tf32": float(d["bf16_tflops"]) * 1.1 / 2.25,
+                "source": "measured (tf32 = measured bf16 x nominal 1.1/2.25)"}
+    return {"hbm": 6650.0, "tf32": 1590.0 * 1.1 / 2.25,
+            "source": "fallback (tf32 = fallback bf16 x nominal 1.1/2.25)"}
+
+
+def route_summary(S, route_ms, peaks):
+    """Rate of the chunk-map step (all maps of one step) against its roofline."""
+    amount, unit, bound = S.route_work()
+    maps = len(S.routers)
+    rate = amount * maps / (route_ms / 1e3) / (1e9 if unit == "GB/s" else 1e12)
+    peak = peaks["hbm"] if bound == "hbm" else peaks["tf32"]
+    out = {"router": S.router, "maps_per_step": maps, "avg_ms_per_step": route_ms,
+           "achieved": rate, "unit": unit, "bound": bound, "peak": peak, "frac": rate / peak,
+           "peak_source": peaks["source"],
+           "algorithmic_per_map": amount, "includes": "map kernels only (layout excluded)"}
+    if bound == "tensor":
+        out["tensor_passes"] = 3   # tf32 hi*hi + hi*lo + lo*hi: 3x the algorithmic MMAs
+    return out
 
 
 # ------------------------------------------------------------------ clocks
@@ -147,7 +177,7 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
 class Setup:
     """Device-resident inputs and outputs of one batch of the workload."""
 
-    def __init__(self, w, seed, device, routing_sharing=True):
+    def __init__(self, w, seed, device, routing_sharing=True, router="moqae"):
         import torch
         from chunk_adaptive_mixed_b200 import mqkv as M
         from chunk_adaptive_mixed_b200 import workloads as W
@@ -166,6 +196,13 @@ class Setup:
         self.routers = [W.router_weights(w, seed + (l if not routing_sharing else 0), device)
                         for l in range(nr)]
         self.W1, self.W2, self.W3, self.b3 = self.routers[0]
+        self.router = router
+        if router == "similarity":
+            # one query vector per sequence (per layer and sequence without
+            # routing sharing); thresholds at the workload's target mix
+            self.u = [W.similarity_query(w, seed + (l if not routing_sharing else 0), device)
+                      for l in range(nr)]
+            self.tau = W.similarity_thresholds(w)
         self.C = W.router_input(w, self.lens, seed, device)
         self.K, self.V, self.q = [], [], []
         for layer in range(w.layers):
@@ -199,9 +236,18 @@ class Setup:
         """One pass of the whole path (launches only; asynchronous)."""
         from chunk_adaptive_mixed_b200 import mqkv as M
         w = self.w
+        if timers:
+            timers["route"][0].record()
         for r, (W1, W2, W3, b3) in enumerate(self.routers):
-            M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, W1, W2, W3, b3,
-                              self.token_expert, self.chunk_experts[r], self.route_ws)
+            if self.router == "similarity":
+                M.mq_similarity_route(self.shape, self.lens, self.cu, self.C, self.u[r],
+                                      self.tau[0], self.tau[1], self.chunk_experts[r])
+            else:
+                M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, W1, W2, W3, b3,
+                                  self.token_expert, self.chunk_experts[r], self.route_ws)
+        if timers:
+            timers["route"][1].record()
+        for r in range(len(self.routers)):
             M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_experts[r],
                               self.layouts[r])
         for layer in range(w.layers):
@@ -224,9 +270,21 @@ class Setup:
         return self.layouts[0 if self.rs else layer]
 
     def launches_per_step(self):
-        # per router: weight split + router + vote and 2 layout kernels; one
-        # pack per layer; two decode kernels per layer and decode step
-        return 5 * len(self.routers) + self.w.layers + 2 * self.w.layers * self.w.decode_steps
+        # per map: weight split + router + vote (or one similarity kernel) and
+        # 2 layout kernels; one pack per layer; two decode kernels per layer
+        # and decode step
+        per_map = 3 if self.router == "similarity" else 5
+        return (per_map * len(self.routers) + self.w.layers
+                + 2 * self.w.layers * self.w.decode_steps)
+
+    def route_work(self):
+        """Algorithmic work of one map: (amount, unit, bound).  The router is
+        two D x H projections per token (the small W3 product aside); the
+        similarity search reads C and u once and writes one byte per chunk."""
+        w = self.w
+        if self.router == "similarity":
+            return (self.T * w.router_dim * 4 + self.B * w.router_dim * 4 + self.N, "GB/s", "hbm")
+        return (4.0 * self.T * w.router_dim * w.router_hidden, "TFLOP/s", "tensor")
 
 
 def run_ours(args, rank, world, local_rank):
@@ -240,7 +298,7 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     w = W.get(args.workload)
     seed = rank_seed(args.seed, rank)
-    S = Setup(w, seed, device, routing_sharing=not args.no_rs)
+    S = Setup(w, seed, device, routing_sharing=not args.no_rs, router=args.router)
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -266,7 +324,8 @@ def run_ours(args, rank, world, local_rank):
     t_start, t_end = E(enable_timing=True), E(enable_timing=True)
     t_start.record()
     for _ in range(args.steps):
-        tm = {"pack": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)],
+        tm = {"route": (E(enable_timing=True), E(enable_timing=True)),
+              "pack": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)],
               "decode": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)]}
         S.step(tm)
         timers_all.append(tm)
@@ -279,6 +338,7 @@ def run_ours(args, rank, world, local_rank):
     ms_step = ms / args.steps
     pack_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["pack"]]
     dec_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["decode"]]
+    route_ms = float(np.mean([tm["route"][0].elapsed_time(tm["route"][1]) for tm in timers_all]))
     pack_avg = float(np.mean(pack_ms))
     dec_avg = float(np.mean(dec_ms))
 
@@ -296,7 +356,7 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(S, args, device)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, S.lens, seed, tokens_per_step)
+        cpu = cpu_baseline(w, S.lens, seed, tokens_per_step, S.router, len(S.routers))
 
     if rank == 0:
         line = {
@@ -310,7 +370,7 @@ def run_ours(args, rank, world, local_rank):
                        "head_dim": w.head_dim, "chunk_len": w.chunk_len,
                        "router_D": w.router_dim, "router_H": w.router_hidden,
                        "kv_dtype": w.kv_dtype, "decode_steps": w.decode_steps,
-                       "routing_sharing": S.rs,
+                       "routing_sharing": S.rs, "router": S.router,
                        "parallelism": f"dp{world} (independent batches)",
                        "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
                        else "inputs fit in L2"},
@@ -323,6 +383,7 @@ def run_ours(args, rank, world, local_rank):
             "decode_attn": {"GB/s": dec_gbs, "frac": dec_gbs / peak, "avg_ms_per_layer": dec_avg,
                             "tokens_per_s_attention_only": S.B / (dec_avg * w.layers / 1e3),
                             "algorithmic_bytes_per_layer": dec_bytes},
+            "route": route_summary(S, route_ms, peaks_all()),
             "pack": {"GB/s": pack_gbs, "frac": pack_gbs / peak, "avg_ms_per_layer": pack_avg},
             "packed_bytes_per_layer": pb,
             "chunk_mix": [round(float(x), 4) for x in mix],
@@ -351,13 +412,16 @@ def run_e2e(S, args, device):
     host["K"] = [pinned_copy(K) for K in S.K]
     host["V"] = [pinned_copy(V) for V in S.V]
     host["q"] = [[pinned_copy(q) for q in qs] for qs in S.q]
+    host["u"] = [pinned_copy(u) for u in S.u] if S.router == "similarity" else []
     out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in S.out]
-    h2d = (host["C"].numel() * 4 + sum(x.numel() * x.element_size() for x in host["K"] + host["V"])
+    h2d = (host["C"].numel() * 4 + sum(u.numel() * 4 for u in host["u"]) + sum(x.numel() * x.element_size() for x in host["K"] + host["V"])
            + sum(q.numel() * q.element_size() for qs in host["q"] for q in qs))
     d2h = sum(o.numel() * o.element_size() for o in out_host) * w.decode_steps
 
     def e2e_step():
         S.C.copy_(host["C"], non_blocking=True)
+        for r, u in enumerate(host["u"]):
+            S.u[r].copy_(u, non_blocking=True)
         for layer in range(w.layers):
             S.K[layer].copy_(host["K"][layer], non_blocking=True)
             S.V[layer].copy_(host["V"][layer], non_blocking=True)
@@ -385,7 +449,8 @@ def run_e2e(S, args, device):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_step_estimate(w, lens, seed, route_chunks=32, pack_tokens=32768):
+def oracle_step_estimate(w, lens, seed, route_chunks=32, pack_tokens=32768, router="moqae",
+                         maps=1):
     """Times the CPU oracle on a bounded sample of one step and scales each
     phase to the full step.  Returns (seconds per full step, sample text, cores)."""
     import torch
@@ -399,10 +464,16 @@ def oracle_step_estimate(w, lens, seed, route_chunks=32, pack_tokens=32768):
     nr = min(route_chunks, N)
     C = W.router_input(w, lens, seed, "cpu", chunk_range=(0, nr)).numpy()
     counts = W.chunk_token_counts(lens, L)[:nr].astype(np.int32)
-    t0 = time.perf_counter()
-    z32, _ = O.router_logits(C, W1, W2, W3, b3)
-    O.vote(counts, L, O.token_argmax(z32), True)
-    t_route = (time.perf_counter() - t0) * T / max(int(counts.sum()), 1)
+    if router == "similarity":
+        u = W.similarity_query(w, seed, "cpu").numpy()[:1]
+        tau_hi, tau_lo = W.similarity_thresholds(w)
+        t0 = time.perf_counter()
+        O.similarity_route(np.array([int(counts.sum())], np.int32), L, C, u, tau_hi, tau_lo)
+    else:
+        t0 = time.perf_counter()
+        z32, _ = O.router_logits(C, W1, W2, W3, b3)
+        O.vote(counts, L, O.token_argmax(z32), True)
+    t_route = (time.perf_counter() - t0) * T / max(int(counts.sum()), 1) * maps
     # packing and decode: 1 layer of the first sequence, capped at pack_tokens
     Tp = int(min(lens[0], pack_tokens))
     lens1 = np.array([Tp], np.int32)
@@ -417,14 +488,14 @@ def oracle_step_estimate(w, lens, seed, route_chunks=32, pack_tokens=32768):
     t0 = time.perf_counter()
     O.decode(w.num_q_heads, w.num_kv_heads, w.head_dim, L, lens1, cmap, packed, q)
     t_dec = (time.perf_counter() - t0) * (T / Tp) * w.layers * w.decode_steps
-    sample = (f"route {int(counts.sum())} tokens, pack + decode {Tp} tokens of 1 layer; "
+    sample = (f"{router} map {int(counts.sum())} tokens (x {maps} maps), pack + decode {Tp} tokens of 1 layer; "
               f"each phase scaled to {T} tokens x {w.layers} layers x {w.decode_steps} "
               f"decode step(s)")
     return t_route + t_pack + t_dec, sample, O.num_threads()
 
 
-def cpu_baseline(w, lens, seed, tokens_per_step):
-    t, sample, cores = oracle_step_estimate(w, lens, seed)
+def cpu_baseline(w, lens, seed, tokens_per_step, router="moqae", maps=1):
+    t, sample, cores = oracle_step_estimate(w, lens, seed, router=router, maps=maps)
     return {"value": tokens_per_step / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": sample, "projected_s_per_step": t}
 
@@ -439,7 +510,8 @@ def run_reference(args, rank, world):
     tokens_per_step = len(lens) * w.decode_steps
     # a smaller sample per step than the cpu_baseline leg, so that K + W
     # steps stay within a few minutes
-    kw = dict(route_chunks=8, pack_tokens=8192)
+    kw = dict(route_chunks=8, pack_tokens=8192, router=args.router,
+              maps=w.layers if args.no_rs else 1)
     for _ in range(args.warmup):
         oracle_step_estimate(w, lens, args.seed, **kw)
     times = []
@@ -455,7 +527,8 @@ def run_reference(args, rank, world):
             "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": {"workload": w.name, "layers": w.layers, "num_seqs": len(lens),
-                       "total_tokens": int(lens.sum()), "parallelism": "rank 0 only"},
+                       "total_tokens": int(lens.sum()), "router": args.router,
+                       "routing_sharing": not args.no_rs, "parallelism": "rank 0 only"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,

@@ -288,6 +288,36 @@ mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
   return MQ_OK;
 }
 
+mq_status mq_similarity_route(const mq_shape* shape, const int32_t* h_seq_lens,
+                              const int64_t* d_cu_seqlens, const float* C, int32_t D,
+                              const float* u, double tau_hi, double tau_lo,
+                              int32_t routing_freeze, uint8_t* chunk_expert, double* similarity,
+                              void* stream) {
+  MQ_TRY(check_shape(shape));
+  int64_t T, N;
+  MQ_TRY(check_lens(shape, h_seq_lens, &T, &N));
+  if (D < 1 || D % 4 != 0) return fail(MQ_ERR_INVALID_ARG, "D must be a positive multiple of 4 (got %d)", D);
+  if (shape->num_seqs > 65535)
+    return fail(MQ_ERR_UNSUPPORTED, "num_seqs must be <= 65535 (got %d)", shape->num_seqs);
+  if (tau_hi != tau_hi || tau_lo != tau_lo) return fail(MQ_ERR_INVALID_ARG, "a threshold is NaN");
+  MQ_NEED_PTR(d_cu_seqlens, "d_cu_seqlens");
+  if (T > 0) MQ_NEED_PTR(C, "C");
+  MQ_NEED_PTR(u, "u");
+  if (N > 0) MQ_NEED_PTR(chunk_expert, "chunk_expert");
+  if (similarity && misaligned(similarity))
+    return fail(MQ_ERR_INVALID_ARG, "similarity is not 16-byte aligned");
+  int64_t max_chunks = 0;
+  for (int b = 0; b < shape->num_seqs; ++b) {
+    const int64_t nb = (h_seq_lens[b] + shape->chunk_len - 1) / shape->chunk_len;
+    max_chunks = nb > max_chunks ? nb : max_chunks;
+  }
+  const cudaError_t err = launch_similarity_route(
+      shape->num_seqs, d_cu_seqlens, shape->chunk_len, max_chunks, C, D, u, tau_hi, tau_lo,
+      routing_freeze, chunk_expert, similarity, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "similarity launch");
+  return MQ_OK;
+}
+
 mq_status mq_build_layout(const mq_shape* shape, const int32_t* h_seq_lens,
                           const int64_t* d_cu_seqlens, const uint8_t* chunk_expert, void* layout,
                           size_t layout_bytes, void* stream) {

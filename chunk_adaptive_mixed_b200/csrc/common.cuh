@@ -114,6 +114,11 @@ cudaError_t launch_finish_vote(int B, const int64_t* cu_seqlens, int L, int64_t 
                                const float4* zpart, int nhb, const float* b3, int routing_freeze,
                                uint8_t* token_expert, float* logits, uint8_t* chunk_expert,
                                cudaStream_t stream);
+// Chunk-level search by chunk-query cosine (fp64), grid (max_chunks, B).
+cudaError_t launch_similarity_route(int B, const int64_t* cu_seqlens, int L, int64_t max_chunks,
+                                    const float* C, int D, const float* u, double tau_hi,
+                                    double tau_lo, int routing_freeze, uint8_t* chunk_expert,
+                                    double* similarity, cudaStream_t stream);
 cudaError_t launch_layout(const mq_shape& s, const int64_t* cu_seqlens, const uint8_t* chunk_expert,
                           int64_t total_chunks, const ItemPolicy& pol, void* layout,
                           unsigned int* status, cudaStream_t stream);

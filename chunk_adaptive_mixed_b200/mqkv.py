@@ -36,7 +36,7 @@ MQ_DEV_INDEX_RANGE = 0x10
 # names of every function include/mqkv.h declares
 EXPORTS = ("mq_status_string", "mq_last_error", "mq_layout_bytes", "mq_packed_bytes_upper_bound",
            "mq_decode_workspace_bytes", "mq_route_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
-           "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc")
+           "mq_similarity_route", "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc")
 
 # size of the scratch array built into the library for mq_decode_attn_noalloc
 MQ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -89,6 +89,9 @@ def lib() -> ctypes.CDLL:
     L.mq_route_chunks.restype = ctypes.c_int
     L.mq_route_chunks.argtypes = [sp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp,
                                   sz, vp]
+    L.mq_similarity_route.restype = ctypes.c_int
+    L.mq_similarity_route.argtypes = [sp, vp, vp, vp, i32, vp, ctypes.c_double, ctypes.c_double,
+                                      i32, vp, vp, vp]
     L.mq_build_layout.restype = ctypes.c_int
     L.mq_build_layout.argtypes = [sp, vp, vp, vp, vp, sz, vp]
     L.mq_pack_kv.restype = ctypes.c_int
@@ -206,6 +209,15 @@ def mq_route_chunks(shp, seq_lens, cu_seqlens, C, W1, W2, W3, b3, token_expert, 
                                  _ptr(W1), _ptr(W2), _ptr(W3), _ptr(b3), int(bool(routing_freeze)),
                                  _ptr(token_expert), _ptr(chunk_expert), _ptr(logits),
                                  _ptr(workspace), nbytes, _stream(stream)), "mq_route_chunks")
+
+
+def mq_similarity_route(shp, seq_lens, cu_seqlens, C, u, tau_hi, tau_lo, chunk_expert,
+                        similarity=None, routing_freeze=True, stream=None):
+    l = _lens(seq_lens)
+    _check(lib().mq_similarity_route(ctypes.byref(shp), l.ctypes.data, _ptr(cu_seqlens), _ptr(C),
+                                     int(C.shape[1]), _ptr(u), float(tau_hi), float(tau_lo),
+                                     int(bool(routing_freeze)), _ptr(chunk_expert),
+                                     _ptr(similarity), _stream(stream)), "mq_similarity_route")
 
 
 def mq_build_layout(shp, seq_lens, cu_seqlens, chunk_expert, layout, stream=None):

@@ -26,7 +26,10 @@ Router input C: tokens of one chunk share a common direction,
 C_t = sqrt(rho) * z_chunk + sqrt(1 - rho) * z_t with z ~ N(0, I) and rho = 0.9,
 so each coordinate is N(0, 1) and chunks differ from one another (with
 independent tokens every chunk would vote alike).  W1, W2 ~ N(0, 1/D),
-W3 ~ N(0, 1/H).  The per-expert bias b3 of each workload is a fixed input that
+W3 ~ N(0, 1/H).  The similarity search takes one query vector per sequence,
+u_b ~ N(0, I), independent of C; the cosine of two independent directions in
+D dimensions is close to N(0, 1/D), so its thresholds are that normal's
+quantiles at the target mix.  The per-expert bias b3 of each workload is a fixed input that
 was chosen offline with the CPU oracle (tests/golden/fit_router_bias.py) so
 that the chunk-level mix lands near the target; the achieved mix is measured
 and reported, never assumed.
@@ -44,7 +47,7 @@ EXPERT_BITS = (16, 4, 2)
 
 # stream tags for seed derivation
 _TAG = {"seq_lens": 1, "c_chunk": 2, "c_token": 3, "w1": 4, "w2": 5, "w3": 6, "k": 7, "v": 8,
-        "q": 9, "outliers": 10, "map": 11}
+        "q": 9, "outliers": 10, "map": 11, "u": 12}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -219,6 +222,22 @@ def router_input(w: Workload, lens: np.ndarray, seed: int = 0, device="cpu",
 
 
 _CHUNK_BLOCK = 64
+
+
+def similarity_query(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
+    """u [B, D] fp32 ~ N(0, I): one query vector per sequence."""
+    return torch.randn(w.num_seqs, w.router_dim, generator=generator(device, seed, _TAG["u"]),
+                       device=device)
+
+
+def similarity_thresholds(w: Workload) -> Tuple[float, float]:
+    """(tau_hi, tau_lo) putting about target_mix of the chunks in FP16 / INT4 /
+    INT2 when the cosine is close to N(0, 1/D) (independent query)."""
+    from statistics import NormalDist
+    f16, _, f2 = w.target_mix
+    sd = 1.0 / np.sqrt(w.router_dim)
+    nd = NormalDist()
+    return float(nd.inv_cdf(1.0 - f16) * sd), float(nd.inv_cdf(f2) * sd)
 
 
 def chunk_token_counts(lens: np.ndarray, L: int) -> np.ndarray:

@@ -9,6 +9,9 @@
  *                    chunk takes the majority choice of its tokens.
  *                    (MoQAE paper notes, 方法详解 › 整体框架 and
  *                     关键设计 › Quantization-Aware Experts.)
+ *   mq_similarity_route  alternative chunk map: each chunk's bitwidth from its
+ *                    similarity to a per-sequence query vector (Cocktail
+ *                    abstract: chunk-level quantization search).
  *   mq_build_layout  chunks of each sequence are regrouped by precision into
  *                    contiguous FP16 → INT4 → INT2 segments before anything is
  *                    quantised (Cocktail abstract on the "Bin Zhang" scholarfeed
@@ -259,6 +262,39 @@ mq_status mq_route_chunks(const mq_shape* shape, const int32_t* h_seq_lens,
                           uint8_t* token_expert, uint8_t* chunk_expert,
                           float* logits, void* workspace, size_t workspace_bytes,
                           void* stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_similarity_route — chunk-level quantization search by similarity, an
+ * alternative to mq_route_chunks that writes the same chunk_expert map.
+ *
+ * Cocktail abstract on the "Bin Zhang" scholarfeed author page: the bitwidth
+ * of each context chunk follows from how similar the chunk is to the query.
+ * The page names neither the similarity nor the cut-offs; this library reads
+ * it as the cosine between the chunk's mean router-input row and a per-
+ * sequence query vector u_b, cut at two thresholds the caller gives:
+ *     m_(b,c) = mean of C_t over the chunk's tokens (a short tail chunk
+ *               averages its own tokens),
+ *     sim     = <m, u_b> / (|m| |u_b|),   0 when either vector is zero,
+ *     expert  = FP16 if sim >= tau_hi, else INT4 if sim >= tau_lo, else INT2.
+ * With routing_freeze != 0, chunk 0 of every sequence is FP16 (the same
+ * freezing rule as the router's).  Sums and the threshold test are in fp64.
+ *
+ *   C            device fp32 [T, D] row-major (rows as for mq_route_chunks)
+ *   u            device fp32 [B, D] row-major, one query vector per sequence
+ *   tau_hi, tau_lo  thresholds (any finite values; tau_hi <= tau_lo makes
+ *                INT4 unreachable)
+ *   chunk_expert device uint8 [N]  out, chunk (b, c) at chunk_offset_b + c
+ *   similarity   device fp64 [N] out, or NULL
+ * Constraints: 1 <= D, D % 4 == 0; B <= 65535.  Needs no workspace.  NaN
+ * thresholds are rejected (MQ_ERR_INVALID_ARG).  A NaN or infinite value in C
+ * or u gives a NaN similarity, which compares false and maps to INT2.
+ * ------------------------------------------------------------------------- */
+mq_status mq_similarity_route(const mq_shape* shape, const int32_t* h_seq_lens,
+                              const int64_t* d_cu_seqlens,
+                              const float* C, int32_t D, const float* u,
+                              double tau_hi, double tau_lo, int32_t routing_freeze,
+                              uint8_t* chunk_expert, double* similarity,
+                              void* stream);
 
 /* ---------------------------------------------------------------------------
  * mq_build_layout — Cocktail's chunk regrouping (chunk-level KV cache

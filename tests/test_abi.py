@@ -143,3 +143,27 @@ def test_size_queries_match_the_format(d, L):
         O.packed_bytes(2, d, L, lens, np.zeros(n, np.uint8))
     ce = rng.integers(0, 3, n).astype(np.uint8)
     assert O.packed_bytes(2, d, L, lens, ce) <= M.mq_packed_bytes_upper_bound(shp, lens)
+
+
+def test_similarity_route_validation():
+    lib = M.lib()
+    shp = _shape()
+    lens = LENS.copy()
+    p = 1 << 20
+    nan = float("nan")
+    f = lib.mq_similarity_route
+    assert f(ctypes.byref(shp), lens.ctypes.data, p, p, 64, p, 0.1, 0.0, 1, p, None, 0) \
+        == M.MQ_ERR_CUDA                                   # valid, but no device here
+    assert f(ctypes.byref(shp), lens.ctypes.data, p, p, 66, p, 0.1, 0.0, 1, p, None, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    assert f(ctypes.byref(shp), lens.ctypes.data, p, p, 64, p, nan, 0.0, 1, p, None, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    assert "NaN" in M.last_error()
+    assert f(ctypes.byref(shp), lens.ctypes.data, p, p, 64, None, 0.1, 0.0, 1, p, None, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    assert f(ctypes.byref(shp), lens.ctypes.data, p, p, 64, p, 0.1, 0.0, 1, p, p + 8, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    big = _shape(num_seqs=70000)
+    many = np.full(70000, 1, np.int32)
+    assert f(ctypes.byref(big), many.ctypes.data, p, p, 64, p, 0.1, 0.0, 1, p, None, 0) \
+        == M.MQ_ERR_UNSUPPORTED

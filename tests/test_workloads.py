@@ -71,3 +71,20 @@ def test_workload_mix_near_target(name, chunks):
     ce = O.vote(counts, int(counts.max()), O.token_argmax(z32), routing_freeze=False)
     mix = np.bincount(ce, minlength=3) / len(ce)
     assert np.abs(mix - np.asarray(w.target_mix)).max() < 0.12, mix
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama2_13b_128k"])
+def test_similarity_thresholds_give_the_target_mix(name):
+    # many sequences of a few chunks each, so the mix is measured over ~256 chunks
+    w = W.scaled(W.get(name), num_seqs=256, seq_len=2 * W.get(name).chunk_len,
+                 seq_len_range=None, router_dim=256)
+    lens = W.seq_lens(w)
+    C = W.router_input(w, lens).numpy()
+    u = W.similarity_query(w).numpy()
+    assert u.shape == (256, 256)
+    tau_hi, tau_lo = W.similarity_thresholds(w)
+    assert tau_hi > tau_lo
+    ce, sim = O.similarity_route(lens, w.chunk_len, C, u, tau_hi, tau_lo, routing_freeze=False)
+    assert abs(sim.std() * np.sqrt(w.router_dim) - 1.0) < 0.15   # cos ~ N(0, 1/D)
+    mix = np.bincount(ce, minlength=3) / len(ce)
+    assert np.abs(mix - np.asarray(w.target_mix)).max() < 0.08, mix
