@@ -49,6 +49,13 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--router", default="moqae", choices=["moqae", "similarity"],
                    help="chunk map from MoQAE's router or from Cocktail's chunk-query similarity")
+    p.add_argument("--layers", type=int, default=0,
+                   help="override the workload's layer count (small profiling cases)")
+    p.add_argument("--seqs", type=int, default=0,
+                   help="override the workload's sequence count (small profiling cases)")
+    p.add_argument("--lam", type=float, default=0.0,
+                   help="memory-pressure knob for the router map: subtracts lam * bits/16 from "
+                        "each expert's bias (more INT2 as lam grows, more FP16 below 0)")
     p.add_argument("--no-rs", action="store_true",
                    help="routing sharing off: one router, map and layout per layer")
     return p.parse_args()
@@ -149,6 +156,18 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ ranks
 
+def workload(args):
+    """The named workload, with the layer / sequence overrides applied."""
+    from chunk_adaptive_mixed_b200 import workloads as W
+    w = W.get(args.workload)
+    ch = {}
+    if args.layers:
+        ch["layers"] = args.layers
+    if args.seqs:
+        ch["num_seqs"] = args.seqs
+    return W.scaled(w, **ch) if ch else w
+
+
 def rank_seed(seed: int, rank: int) -> int:
     """Each rank draws its own batch: independent problems, no exchange."""
     return seed + 1009 * rank
@@ -177,7 +196,7 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
 class Setup:
     """Device-resident inputs and outputs of one batch of the workload."""
 
-    def __init__(self, w, seed, device, routing_sharing=True, router="moqae"):
+    def __init__(self, w, seed, device, routing_sharing=True, router="moqae", lam=0.0):
         import torch
         from chunk_adaptive_mixed_b200 import mqkv as M
         from chunk_adaptive_mixed_b200 import workloads as W
@@ -195,6 +214,13 @@ class Setup:
         nr = 1 if routing_sharing else w.layers
         self.routers = [W.router_weights(w, seed + (l if not routing_sharing else 0), device)
                         for l in range(nr)]
+        self.lam = lam
+        if lam:
+            # MoQAE trades accuracy for memory with a weight lambda on the
+            # memory term; at inference the same pressure is a bias against
+            # the wider experts
+            pen = torch.tensor([16.0, 4.0, 2.0], device=device) / 16.0 * lam
+            self.routers = [(W1, W2, W3, b3 - pen) for W1, W2, W3, b3 in self.routers]
         self.W1, self.W2, self.W3, self.b3 = self.routers[0]
         self.router = router
         if router == "similarity":
@@ -296,9 +322,11 @@ def run_ours(args, rank, world, local_rank):
     M.lib()
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
-    w = W.get(args.workload)
+    w = workload(args)
     seed = rank_seed(args.seed, rank)
-    S = Setup(w, seed, device, routing_sharing=not args.no_rs, router=args.router)
+    if args.lam and args.router != "moqae":
+        raise SystemExit("--lam applies to the MoQAE router only")
+    S = Setup(w, seed, device, routing_sharing=not args.no_rs, router=args.router, lam=args.lam)
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -370,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
                        "head_dim": w.head_dim, "chunk_len": w.chunk_len,
                        "router_D": w.router_dim, "router_H": w.router_hidden,
                        "kv_dtype": w.kv_dtype, "decode_steps": w.decode_steps,
-                       "routing_sharing": S.rs, "router": S.router,
+                       "routing_sharing": S.rs, "router": S.router, "lam": S.lam,
                        "parallelism": f"dp{world} (independent batches)",
                        "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
                        else "inputs fit in L2"},
@@ -505,7 +533,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     from chunk_adaptive_mixed_b200 import workloads as W
-    w = W.get(args.workload)
+    w = workload(args)
     lens = W.seq_lens(w, args.seed)
     tokens_per_step = len(lens) * w.decode_steps
     # a smaller sample per step than the cpu_baseline leg, so that K + W

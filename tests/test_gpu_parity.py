@@ -214,3 +214,56 @@ def test_routing_sharing_off_gives_each_layer_its_own_map_and_layout():
         else:
             assert exempt > 0
     assert any(not np.array_equal(maps[0], m) for m in maps[1:])
+
+
+def _adversarial_groups(n_groups, dtype, rng):
+    """Groups of 32 values chosen where an encoder goes wrong: signed zeros as
+    the minimum in either order, constant groups (s = 1), fp16 subnormals,
+    the largest finite fp16 values, and groups whose scaled values sit exactly
+    on half-integers (round-half-even) or one ulp away from them."""
+    g = np.empty((n_groups, 32), np.float32)
+    for i in range(n_groups):
+        kind = i % 8
+        if kind == 0:                                   # zero minimum, -0 first or +0 first
+            x = rng.uniform(0, 3, 32).astype(np.float32)
+            j0, j1 = rng.choice(32, 2, replace=False)
+            x[j0], x[j1] = (-0.0, 0.0) if i % 16 == 0 else (0.0, -0.0)
+        elif kind == 1:                                 # constant group
+            x = np.full(32, rng.choice([0.0, -0.0, 1.5, -7.25]), np.float32)
+        elif kind == 2:                                 # fp16 subnormals and zero
+            x = (rng.integers(-1023, 1024, 32) * 2.0 ** -24).astype(np.float32)
+        elif kind == 3:                                 # extremes of fp16
+            x = rng.choice([-65504.0, 65504.0, -1.0, 0.5, 6.1e-5], 32).astype(np.float32)
+        elif kind in (4, 5):                            # half-way ties at s = 1 (INT4) / s = 1 (INT2)
+            top = 15.0 if kind == 4 else 3.0
+            x = (rng.integers(0, int(top), 32) + 0.5).astype(np.float32)
+            x[0], x[1] = 0.0, top
+        elif kind == 6:                                 # ties at a power-of-two scale
+            x = ((rng.integers(0, 30, 32) + 0.5) * 0.25 - 4.0).astype(np.float32)
+            x[0], x[1] = -4.0, -4.0 + 7.5
+        else:                                           # plain normal values
+            x = rng.standard_normal(32).astype(np.float32)
+        g[i] = x
+    if dtype == "f16":
+        g = g.astype(np.float16).astype(np.float32)     # exactly representable inputs
+    return g
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_pack_adversarial_values_bit_exact(dtype):
+    case = Case(np.array([300, 64, 517], np.int32), 8, 4, 128, 32, dtype)
+    rng = np.random.default_rng(42 if dtype == "f16" else 43)
+    n = case.T * case.Hkv * case.d // 32
+    K = _adversarial_groups(n, dtype, rng).reshape(case.T, case.Hkv, case.d)
+    V = _adversarial_groups(n, dtype, rng)[::-1].copy().reshape(case.T, case.Hkv, case.d)
+    Kt = torch.from_numpy(K).to(case.torch_dtype)
+    Vt = torch.from_numpy(V).to(case.torch_dtype)
+    for mapname, mix in MAPS.items():
+        cmap = _map(case, mix, seed=7)
+        layout = gpu_layout(case, cmap)
+        packed, pb = gpu_pack(case, layout, Kt.to(dev()), Vt.to(dev()))
+        ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, Kt.numpy(), Vt.numpy())
+        got = packed[:pb].cpu().numpy()
+        if not np.array_equal(got, ref):
+            bad = np.nonzero(got != ref)[0]
+            raise AssertionError(f"{mapname}: {len(bad)} packed bytes differ, first at {bad[:8]}")
