@@ -70,6 +70,35 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+# DRAM bytes (read + write) of one full-size pack launch of the default
+# workload, from an ncu capture (the command and counters are recorded under
+# profiles/), valid only for the pack sources with this SHA-256.
+PACK_TRAFFIC = {"workload": "llama2_7b_32l",
+                "sha256": "332f50ffc4a4f93ce6f1023404735377cbc393833f092325753fdb852f05c186",
+                "bytes_per_launch": 2154973952 + 856188416}
+
+
+def pack_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("pack.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "chunk_adaptive_mixed_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def pack_traffic(w, S, seed):
+    """Measured DRAM bytes per pack launch, or None when the capture does not
+    describe this kernel and workload."""
+    from chunk_adaptive_mixed_b200 import workloads as W
+    if (PACK_TRAFFIC["sha256"] is None or w.name != PACK_TRAFFIC["workload"] or seed != 0
+            or w.num_seqs != W.get(w.name).num_seqs or S.router != "moqae" or S.lam
+            or not S.rs):
+        return None
+    return PACK_TRAFFIC["bytes_per_launch"] if pack_sources_sha256() == PACK_TRAFFIC["sha256"] \
+        else None
+
+
 def peaks_all():
     """{hbm GB/s, tf32 TFLOP/s}: the measured copy bandwidth, and the measured
     bf16 GEMM burst rate times the nominal dense tf32/bf16 ratio (1.1 / 2.25)."""
@@ -404,7 +433,7 @@ def run_ours(args, rank, world, local_rank):
                        else "inputs fit in L2"},
             "roofline": {"bound": "hbm", "kernel": "pack_kernel",
                          "achieved": pack_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": pack_gbs / peak, "traffic": None,
+                         "frac": pack_gbs / peak, "traffic": pack_traffic(w, S, seed),
                          "peak_source": peak_kind,
                          "algorithmic_bytes_per_launch": pack_bytes,
                          "avg_launch_ms": pack_avg},

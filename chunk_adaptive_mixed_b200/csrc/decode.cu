@@ -10,18 +10,23 @@
 // regrouped by precision, every stretch of work below reads one precision
 // only — no per-token branching between bitwidths.
 //
-// decode_partial_kernel — persistent CTAs walk the work items of the layout's
-// schedule.  A work item is (sequence b, segment s, kv-head g, token range of
-// at most item_tokens[s] tokens); its four byte ranges (K codes, K scales,
-// V codes, V scales) are staged into shared memory with 1-D TMA bulk copies
-// completing on an mbarrier.  Then, for the Hq/Hkv query heads of g:
-//   scores: one thread per (token, group of 32 dims); the group's dot product
-//           uses the raw codes, dequantisation folded in per group:
-//           q . khat = s * (q . code) + min * sum(q)
-//   softmax: per head max / exp2 / sum over the item (log2 domain)
-//   values:  one thread per (token lane, 8-dim slice); accumulates p*s*code
-//           and p*min per group, reduced across token lanes in shared memory
-//   partial: (m, l, acc[d]) per head to the workspace.
+// decode_partial_kernel — every warp is an independent persistent worker
+// that takes work items w = warp id, warp id + total warps, ...  A work item is
+// (sequence b, segment s, kv-head g, token range of at most item_tokens[s]
+// tokens).  The warp streams the item's four byte ranges (K codes, V codes, K
+// scales, V scales) through its own 4-stage cp.async ring in shared memory,
+// one tile of TPW tokens per stage, every lane copying 16-byte units so each
+// instruction reads whole sectors.  Per tile:
+//   lanes: LPT lanes cover one token (SL dims each), TPW tokens per tile; the
+//          lane keeps its SL query values of all Hq/Hkv heads in registers
+//   scores: q . code on the raw codes (expanded with one byte-permute and a
+//          mask per value pair, see spread_byte), dequantisation folded in per
+//          group: q . khat = s * (q . code) + min * sum(q); shuffle-reduced
+//          over the token's LPT lanes
+//   softmax: online, log2 domain, with a lazily moved reference maximum
+//   values: acc += (p * s) * code per value pair and bias += p * min per head
+//   end of item: the TPW token lanes are merged with shuffles and (m, l,
+//          acc[d]) of every head goes to the workspace.
 // decode_combine_kernel — one warp per (b, query head) merges the partials of
 // all items of (b, g) with the usual max-rescaling.
 #include "common.cuh"
