@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -56,6 +57,9 @@ cudaError_t status_word(unsigned int** out) {
   return cudaSuccess;
 }
 
+// Longest sequence (so that one (K|V, kv-head) region stays below 2^31 bytes).
+constexpr int32_t kMaxSeqTokens = 1 << 23;
+
 mq_status check_shape(const mq_shape* s) {
   if (!s) return fail(MQ_ERR_INVALID_ARG, "shape is NULL");
   if (s->num_seqs < 1) return fail(MQ_ERR_INVALID_ARG, "num_seqs must be >= 1 (got %d)", s->num_seqs);
@@ -84,6 +88,9 @@ mq_status check_lens(const mq_shape* s, const int32_t* h_seq_lens, int64_t* T, i
   int64_t t = 0, n = 0;
   for (int b = 0; b < s->num_seqs; ++b) {
     if (h_seq_lens[b] < 0) return fail(MQ_ERR_INVALID_ARG, "h_seq_lens[%d] < 0", b);
+    if (h_seq_lens[b] > kMaxSeqTokens)
+      return fail(MQ_ERR_UNSUPPORTED, "h_seq_lens[%d] = %d exceeds %d tokens", b, h_seq_lens[b],
+                  kMaxSeqTokens);
     t += h_seq_lens[b];
     n += (h_seq_lens[b] + s->chunk_len - 1) / s->chunk_len;
   }
@@ -160,9 +167,41 @@ int64_t max_items_per_kv_head(const mq_shape& s, const int32_t* h_seq_lens, cons
   return n;
 }
 
+// Growable layouts: lengths the layout is sized for (prefill + growth budget).
+struct GrowDims {
+  std::vector<int32_t> cap_lens;  // h_seq_lens[b] + grow_tokens
+  int grow_chunks;                // chunks that can complete during growth
+  int64_t slots;                  // chunk slots (perm / inv entries)
+};
+
 }  // namespace mqkv
 
 using namespace mqkv;
+
+namespace {
+
+mq_status grow_dims(const mq_shape* shape, const int32_t* h_seq_lens, int32_t grow_tokens,
+                    GrowDims* g, int64_t* T, int64_t* N) {
+  MQ_TRY(check_shape(shape));
+  MQ_TRY(check_lens(shape, h_seq_lens, T, N));
+  if (grow_tokens < 0 || grow_tokens > kMaxSeqTokens)
+    return fail(MQ_ERR_INVALID_ARG, "grow_tokens must be in [0, %d] (got %d)", kMaxSeqTokens,
+                grow_tokens);
+  g->cap_lens.resize(shape->num_seqs);
+  for (int b = 0; b < shape->num_seqs; ++b) {
+    const int64_t c = (int64_t)h_seq_lens[b] + grow_tokens;
+    if (c > kMaxSeqTokens)
+      return fail(MQ_ERR_UNSUPPORTED, "h_seq_lens[%d] + grow_tokens exceeds %d tokens", b,
+                  kMaxSeqTokens);
+    g->cap_lens[b] = (int32_t)c;
+  }
+  g->grow_chunks = (grow_tokens + shape->chunk_len - 1) / shape->chunk_len;
+  g->slots = *N + (int64_t)shape->num_seqs * (g->grow_chunks + 1);
+  if (g->slots >= (int64_t(1) << 31)) return fail(MQ_ERR_UNSUPPORTED, "more than 2^31 chunk slots");
+  return MQ_OK;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -334,7 +373,7 @@ mq_status mq_build_layout(const mq_shape* shape, const int32_t* h_seq_lens,
   cudaError_t err = status_word(&status);
   if (err != cudaSuccess) return cuda_fail(err, "device status word");
   const ItemPolicy p = item_policy(*shape, h_seq_lens);
-  err = launch_layout(*shape, d_cu_seqlens, chunk_expert, N, p, layout, status,
+  err = launch_layout(*shape, d_cu_seqlens, chunk_expert, N, p, -1, layout, status,
                       static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "layout launch");
   return MQ_OK;
@@ -388,6 +427,134 @@ mq_status mq_decode_attn(const mq_shape* shape, const int32_t* h_seq_lens, const
   err = launch_decode(*shape, items, layout, packed, q, q_dtype, softmax_scale, out, workspace,
                       workspace_bytes, status, static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return cuda_fail(err, "decode launch");
+  return MQ_OK;
+}
+
+// ---------------------------------------------------------------- growth
+
+mq_status mq_grow_sizes(const mq_shape* shape, const int32_t* h_seq_lens, int32_t grow_tokens,
+                        size_t* layout_bytes, size_t* packed_bytes_upper_bound,
+                        size_t* decode_workspace_bytes) {
+  GrowDims g;
+  int64_t T, N;
+  MQ_TRY(grow_dims(shape, h_seq_lens, grow_tokens, &g, &T, &N));
+  const int L = shape->chunk_len, d = shape->head_dim, Hkv = shape->num_kv_heads;
+  if (layout_bytes) *layout_bytes = layout_total_bytes(shape->num_seqs, g.slots);
+  if (packed_bytes_upper_bound) {
+    // every present chunk at FP16, plus the growth rows of all three segments
+    uint64_t total = 0;
+    for (int b = 0; b < shape->num_seqs; ++b) {
+      const uint64_t nb = (h_seq_lens[b] + L - 1) / L;
+      for (int e = 0; e < kNumExperts; ++e) {
+        const uint64_t rows = ((e == 0 ? nb + 1 : 0) + g.grow_chunks) * (uint64_t)L;
+        uint64_t rb = align128(rows * code_row_bytes(d, e));
+        if (e != 0) rb += align128(rows * scale_row_bytes(d));
+        total += 2ull * Hkv * rb;
+      }
+    }
+    *packed_bytes_upper_bound = total;
+  }
+  if (decode_workspace_bytes) {
+    const ItemPolicy p = item_policy(*shape, g.cap_lens.data());
+    *decode_workspace_bytes =
+        mqkv::decode_workspace_bytes(*shape, max_items_per_kv_head(*shape, g.cap_lens.data(), p));
+  }
+  return MQ_OK;
+}
+
+mq_status mq_grow_build_layout(const mq_shape* shape, const int32_t* h_seq_lens,
+                               int32_t grow_tokens, const int64_t* d_cu_seqlens,
+                               const uint8_t* chunk_expert, void* layout, size_t layout_bytes,
+                               void* stream) {
+  GrowDims g;
+  int64_t T, N;
+  MQ_TRY(grow_dims(shape, h_seq_lens, grow_tokens, &g, &T, &N));
+  MQ_NEED_PTR(d_cu_seqlens, "d_cu_seqlens");
+  if (N > 0) MQ_NEED_PTR(chunk_expert, "chunk_expert");
+  MQ_NEED_PTR(layout, "layout");
+  const size_t need = layout_total_bytes(shape->num_seqs, g.slots);
+  if (layout_bytes < need)
+    return fail(MQ_ERR_WORKSPACE, "layout_bytes %zu < %zu needed", layout_bytes, need);
+  unsigned int* status = nullptr;
+  cudaError_t err = status_word(&status);
+  if (err != cudaSuccess) return cuda_fail(err, "device status word");
+  const ItemPolicy p = item_policy(*shape, g.cap_lens.data());
+  err = launch_layout(*shape, d_cu_seqlens, chunk_expert, g.slots, p, g.grow_chunks, layout,
+                      status, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "layout launch");
+  return MQ_OK;
+}
+
+mq_status mq_grow_pack_kv(const mq_shape* shape, const int32_t* h_seq_lens, int32_t grow_tokens,
+                          const void* layout, const void* K, const void* V, int32_t kv_dtype,
+                          void* packed, size_t packed_bytes, void* stream) {
+  GrowDims g;
+  int64_t T, N;
+  MQ_TRY(grow_dims(shape, h_seq_lens, grow_tokens, &g, &T, &N));
+  if (kv_dtype != MQ_F16 && kv_dtype != MQ_F32)
+    return fail(MQ_ERR_INVALID_ARG, "kv_dtype must be MQ_F16 or MQ_F32 (got %d)", kv_dtype);
+  MQ_NEED_PTR(layout, "layout");
+  MQ_NEED_PTR(packed, "packed");
+  if (T > 0) {
+    MQ_NEED_PTR(K, "K");
+    MQ_NEED_PTR(V, "V");
+  }
+  unsigned int* status = nullptr;
+  cudaError_t err = status_word(&status);
+  if (err != cudaSuccess) return cuda_fail(err, "device status word");
+  err = launch_pack(*shape, g.slots, layout, K, V, kv_dtype, packed, packed_bytes, status,
+                    static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "pack launch");
+  return MQ_OK;
+}
+
+mq_status mq_grow_commit(const mq_shape* shape, void* layout, const uint8_t* sealed,
+                         int32_t add_token, void* stream) {
+  MQ_TRY(check_shape(shape));
+  MQ_NEED_PTR(layout, "layout");
+  if (sealed && misaligned(sealed)) return fail(MQ_ERR_INVALID_ARG, "sealed is not 16-byte aligned");
+  if (add_token != 0 && add_token != 1)
+    return fail(MQ_ERR_INVALID_ARG, "add_token must be 0 or 1 (got %d)", add_token);
+  unsigned int* status = nullptr;
+  cudaError_t err = status_word(&status);
+  if (err != cudaSuccess) return cuda_fail(err, "device status word");
+  err = launch_grow_commit(*shape, sealed, add_token, layout, status,
+                           static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "grow commit launch");
+  return MQ_OK;
+}
+
+mq_status mq_grow_append_kv(const mq_shape* shape, const void* layout, const void* K_new,
+                            const void* V_new, int32_t kv_dtype, void* packed,
+                            size_t packed_bytes, void* stream) {
+  MQ_TRY(check_shape(shape));
+  if (kv_dtype != MQ_F16 && kv_dtype != MQ_F32)
+    return fail(MQ_ERR_INVALID_ARG, "kv_dtype must be MQ_F16 or MQ_F32 (got %d)", kv_dtype);
+  MQ_NEED_PTR(layout, "layout");
+  MQ_NEED_PTR(K_new, "K_new");
+  MQ_NEED_PTR(V_new, "V_new");
+  MQ_NEED_PTR(packed, "packed");
+  unsigned int* status = nullptr;
+  cudaError_t err = status_word(&status);
+  if (err != cudaSuccess) return cuda_fail(err, "device status word");
+  err = launch_grow_append(*shape, layout, K_new, V_new, kv_dtype, packed, packed_bytes, status,
+                           static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "grow append launch");
+  return MQ_OK;
+}
+
+mq_status mq_grow_seal(const mq_shape* shape, const void* layout, const uint8_t* sealed,
+                       void* packed, size_t packed_bytes, void* stream) {
+  MQ_TRY(check_shape(shape));
+  MQ_NEED_PTR(layout, "layout");
+  MQ_NEED_PTR(sealed, "sealed");
+  MQ_NEED_PTR(packed, "packed");
+  unsigned int* status = nullptr;
+  cudaError_t err = status_word(&status);
+  if (err != cudaSuccess) return cuda_fail(err, "device status word");
+  err = launch_grow_seal(*shape, layout, sealed, packed, packed_bytes, status,
+                         static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "grow seal launch");
   return MQ_OK;
 }
 

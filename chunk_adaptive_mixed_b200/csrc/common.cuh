@@ -119,9 +119,20 @@ cudaError_t launch_similarity_route(int B, const int64_t* cu_seqlens, int L, int
                                     const float* C, int D, const float* u, double tau_hi,
                                     double tau_lo, int routing_freeze, uint8_t* chunk_expert,
                                     double* similarity, cudaStream_t stream);
+// grow < 0: fixed layout over total_slots = N chunks; grow >= 0: growable,
+// total_slots = N + B * (grow + 1).
 cudaError_t launch_layout(const mq_shape& s, const int64_t* cu_seqlens, const uint8_t* chunk_expert,
-                          int64_t total_chunks, const ItemPolicy& pol, void* layout,
+                          int64_t total_slots, const ItemPolicy& pol, int grow, void* layout,
                           unsigned int* status, cudaStream_t stream);
+// Growth steps of a growable layout (sealed: device uint8[B] or NULL).
+cudaError_t launch_grow_commit(const mq_shape& s, const uint8_t* sealed, int add, void* layout,
+                               unsigned int* status, cudaStream_t stream);
+cudaError_t launch_grow_seal(const mq_shape& s, const void* layout, const uint8_t* sealed,
+                             void* packed, uint64_t packed_bytes, unsigned int* status,
+                             cudaStream_t stream);
+cudaError_t launch_grow_append(const mq_shape& s, const void* layout, const void* K_new,
+                               const void* V_new, int kv_dtype, void* packed,
+                               uint64_t packed_bytes, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_pack(const mq_shape& s, int64_t total_chunks, const void* layout, const void* K,
                         const void* V, int kv_dtype, void* packed, uint64_t packed_bytes,
                         unsigned int* status, cudaStream_t stream);

@@ -32,11 +32,16 @@ MQ_DEV_WORKSPACE_TOO_SMALL = 0x2
 MQ_DEV_BAD_LAYOUT = 0x4
 MQ_DEV_WAIT_TIMEOUT = 0x8
 MQ_DEV_INDEX_RANGE = 0x10
+MQ_DEV_CAPACITY = 0x20
+MQ_GROW_OPEN = 0x1
+MQ_GROW_FULL = 0x2
 
 # names of every function include/mqkv.h declares
 EXPORTS = ("mq_status_string", "mq_last_error", "mq_layout_bytes", "mq_packed_bytes_upper_bound",
            "mq_decode_workspace_bytes", "mq_route_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
-           "mq_similarity_route", "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc")
+           "mq_similarity_route", "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc",
+           "mq_grow_sizes", "mq_grow_build_layout", "mq_grow_pack_kv", "mq_grow_commit",
+           "mq_grow_append_kv", "mq_grow_seal")
 
 # size of the scratch array built into the library for mq_decode_attn_noalloc
 MQ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -94,6 +99,19 @@ def lib() -> ctypes.CDLL:
                                       i32, vp, vp, vp]
     L.mq_build_layout.restype = ctypes.c_int
     L.mq_build_layout.argtypes = [sp, vp, vp, vp, vp, sz, vp]
+    szp = ctypes.POINTER(ctypes.c_size_t)
+    L.mq_grow_sizes.restype = ctypes.c_int
+    L.mq_grow_sizes.argtypes = [sp, vp, i32, szp, szp, szp]
+    L.mq_grow_build_layout.restype = ctypes.c_int
+    L.mq_grow_build_layout.argtypes = [sp, vp, i32, vp, vp, vp, sz, vp]
+    L.mq_grow_pack_kv.restype = ctypes.c_int
+    L.mq_grow_pack_kv.argtypes = [sp, vp, i32, vp, vp, vp, i32, vp, sz, vp]
+    L.mq_grow_commit.restype = ctypes.c_int
+    L.mq_grow_commit.argtypes = [sp, vp, vp, i32, vp]
+    L.mq_grow_append_kv.restype = ctypes.c_int
+    L.mq_grow_append_kv.argtypes = [sp, vp, vp, vp, i32, vp, sz, vp]
+    L.mq_grow_seal.restype = ctypes.c_int
+    L.mq_grow_seal.argtypes = [sp, vp, vp, vp, sz, vp]
     L.mq_pack_kv.restype = ctypes.c_int
     L.mq_pack_kv.argtypes = [sp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.mq_decode_attn.restype = ctypes.c_int
@@ -252,3 +270,49 @@ def mq_decode_attn_noalloc(shp, seq_lens, layout, packed, q, out, softmax_scale=
                                         _ptr(packed), _ptr(q), _dtype_code(q),
                                         float(softmax_scale), _ptr(out), _stream(stream)),
            "mq_decode_attn_noalloc")
+
+
+# ------------------------------------------------------------------ growth
+
+def mq_grow_sizes(shp, seq_lens, grow_tokens):
+    """(layout bytes, packed-bytes upper bound, decode workspace bytes)."""
+    l = _lens(seq_lens)
+    a, b, c = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib().mq_grow_sizes(ctypes.byref(shp), l.ctypes.data, int(grow_tokens),
+                               ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)), "mq_grow_sizes")
+    return a.value, b.value, c.value
+
+
+def mq_grow_build_layout(shp, seq_lens, grow_tokens, cu_seqlens, chunk_expert, layout,
+                         stream=None):
+    l = _lens(seq_lens)
+    nbytes = layout.numel() * layout.element_size()
+    _check(lib().mq_grow_build_layout(ctypes.byref(shp), l.ctypes.data, int(grow_tokens),
+                                      _ptr(cu_seqlens), _ptr(chunk_expert), _ptr(layout), nbytes,
+                                      _stream(stream)), "mq_grow_build_layout")
+
+
+def mq_grow_pack_kv(shp, seq_lens, grow_tokens, layout, K, V, packed, stream=None):
+    l = _lens(seq_lens)
+    nbytes = packed.numel() * packed.element_size()
+    _check(lib().mq_grow_pack_kv(ctypes.byref(shp), l.ctypes.data, int(grow_tokens), _ptr(layout),
+                                 _ptr(K), _ptr(V), _dtype_code(K), _ptr(packed), nbytes,
+                                 _stream(stream)), "mq_grow_pack_kv")
+
+
+def mq_grow_commit(shp, layout, sealed=None, add_token=True, stream=None):
+    _check(lib().mq_grow_commit(ctypes.byref(shp), _ptr(layout), _ptr(sealed),
+                                int(bool(add_token)), _stream(stream)), "mq_grow_commit")
+
+
+def mq_grow_append_kv(shp, layout, K_new, V_new, packed, stream=None):
+    nbytes = packed.numel() * packed.element_size()
+    _check(lib().mq_grow_append_kv(ctypes.byref(shp), _ptr(layout), _ptr(K_new), _ptr(V_new),
+                                   _dtype_code(K_new), _ptr(packed), nbytes, _stream(stream)),
+           "mq_grow_append_kv")
+
+
+def mq_grow_seal(shp, layout, sealed, packed, stream=None):
+    nbytes = packed.numel() * packed.element_size()
+    _check(lib().mq_grow_seal(ctypes.byref(shp), _ptr(layout), _ptr(sealed), _ptr(packed), nbytes,
+                              _stream(stream)), "mq_grow_seal")

@@ -20,6 +20,8 @@
  *                    and written into those segments.
  *   mq_decode_attn   single-query attention for every sequence, read directly
  *                    from the mixed-bitwidth packed cache.
+ *   mq_grow_*        decode-time growth: new tokens in an FP16 tail, each full
+ *                    chunk routed and appended to its precision segment.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -142,6 +144,7 @@ typedef struct mq_shape {
 #define MQ_DEV_BAD_LAYOUT         0x4u  /* layout magic/shape mismatch */
 #define MQ_DEV_WAIT_TIMEOUT       0x8u  /* a bounded wait on a copy gave up */
 #define MQ_DEV_INDEX_RANGE        0x10u /* an index left its valid range */
+#define MQ_DEV_CAPACITY           0x20u /* a growth step exceeded a reserved capacity */
 
 /* ---------------------------------------------------------------------------
  * Layout table (device memory written by mq_build_layout; part of this ABI).
@@ -171,7 +174,8 @@ typedef struct mq_layout_header {
   int64_t  total_tokens;    /* T */
   uint64_t packed_bytes;    /* bytes of one layer's packed buffer */
   int32_t  item_tokens[3];  /* schedule: max tokens of a work item, per segment */
-  int32_t  reserved[1];     /* zero */
+  int32_t  grow_chunks;     /* 0: fixed layout; > 0: growable (mq_grow_*), chunk
+                               slots per sequence beyond its built chunks */
 } mq_layout_header;         /* 64 bytes */
 
 typedef struct mq_seq_layout {
@@ -187,8 +191,14 @@ typedef struct mq_seq_layout {
   uint64_t scale_offset[3];   /* byte offset of scales inside an INT region (0 for FP16) */
   int32_t  item_begin[3];     /* schedule: first work item of (b, s) */
   int32_t  item_count[3];     /* schedule: work items of (b, s) */
-  int32_t  reserved[2];       /* zero */
+  int32_t  chunk_capacity;    /* growable: chunk slots of b (perm/inv entries
+                                 reserved at chunk_offset); fixed: 0 */
+  int32_t  grow_state;        /* growable: MQ_GROW_* bits; fixed: 0 */
 } mq_seq_layout;              /* 160 bytes */
+
+/* grow_state bits */
+#define MQ_GROW_OPEN 0x1  /* the last chunk is the open FP16 tail (not yet routed) */
+#define MQ_GROW_FULL 0x2  /* the last growth step found no room for this sequence */
 
 /* ---------------------------------------------------------------------------
  * Status and sizes
@@ -378,6 +388,96 @@ mq_status mq_decode_attn_noalloc(const mq_shape* shape, const int32_t* h_seq_len
                                  const void* layout, const void* packed,
                                  const void* q, int32_t q_dtype, float softmax_scale,
                                  float* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Cache growth during decoding (mq_grow_*).
+ *
+ * The pages describe routing and packing of a prefilled context and say
+ * nothing about tokens produced while decoding; this library follows the
+ * plain reading that new tokens accumulate in an FP16 tail and that a chunk
+ * is routed, quantised and appended to its precision segment once it holds L
+ * tokens (MoQAE notes, 整体框架: one bitwidth per chunk; Cocktail abstract:
+ * chunks grouped by precision).
+ *
+ * A growable layout reserves, per sequence, room for `grow_tokens` more
+ * tokens: ceil(grow_tokens / L) more chunks in every segment (the FP16
+ * segment one more, for the open tail) and as many chunk slots in perm/inv.
+ * The last chunk of a sequence, when partial, is the OPEN tail: it is kept in
+ * FP16 at the end of the FP16 segment whatever chunk_expert says, and it is
+ * the only partial chunk.  Each decode step, in this order:
+ *
+ *   mq_grow_commit(layout, sealed, 1)        once: applies the seals of the
+ *                                            previous step, then reserves one
+ *                                            token row per sequence
+ *   for every layer:
+ *     mq_grow_append_kv(layout, K_new, V_new, packed[layer])
+ *     mq_decode_attn(h_seq_lens + grow_tokens, layout, packed[layer], q, ...)
+ *   if some sequence's open tail now holds L tokens:
+ *     route it (mq_route_chunks or mq_similarity_route over its L rows, with
+ *     routing_freeze only for a sequence's chunk 0) into sealed[B]
+ *     (255 = no seal for that sequence)
+ *     for every layer: mq_grow_seal(layout, sealed, packed[layer])
+ *
+ * mq_grow_seal encodes the full tail from its fp16 rows into the next free
+ * rows of segment sealed[b] (1 or 2; 0 leaves it in FP16); the following
+ * mq_grow_commit moves the chunk there in the layout (perm, inv, counts,
+ * decode schedule).  Every step touches O(L) rows per layer.  The result is
+ * the layout and packed bytes that mq_build_layout / mq_pack_kv would give
+ * for the grown sequences with the same map, except that (a) regions keep
+ * their reserved capacity, and (b) chunks quantised from the tail were
+ * quantised from fp16 values (the tail's storage), which matters only for
+ * fp32 inputs.  A step that would overflow a reservation is skipped for that
+ * sequence, sets MQ_GROW_FULL in its grow_state and MQ_DEV_CAPACITY in the
+ * status word.  All calls are asynchronous on `stream`; none synchronises.
+ * ------------------------------------------------------------------------- */
+
+/* Sizes for a growable layout: layout table bytes, an upper bound of one
+ * layer's packed bytes (every present chunk at FP16 plus all reservations),
+ * and the decode workspace for the grown lengths.  Output pointers may be
+ * NULL.  Constraints as mq_build_layout, 0 <= grow_tokens and every
+ * h_seq_lens[b] + grow_tokens <= 2^23. */
+mq_status mq_grow_sizes(const mq_shape* shape, const int32_t* h_seq_lens,
+                        int32_t grow_tokens, size_t* layout_bytes,
+                        size_t* packed_bytes_upper_bound,
+                        size_t* decode_workspace_bytes);
+
+/* mq_build_layout for a growable layout (header.grow_chunks > 0).  The
+ * chunk_expert entry of a partial last chunk is ignored (open tail, FP16). */
+mq_status mq_grow_build_layout(const mq_shape* shape, const int32_t* h_seq_lens,
+                               int32_t grow_tokens, const int64_t* d_cu_seqlens,
+                               const uint8_t* chunk_expert, void* layout,
+                               size_t layout_bytes, void* stream);
+
+/* mq_pack_kv for a growable layout (same arguments plus grow_tokens, which
+ * must be the value the layout was built with); packed must hold
+ * header.packed_bytes (mq_packed_bytes). */
+mq_status mq_grow_pack_kv(const mq_shape* shape, const int32_t* h_seq_lens,
+                          int32_t grow_tokens, const void* layout, const void* K,
+                          const void* V, int32_t kv_dtype, void* packed,
+                          size_t packed_bytes, void* stream);
+
+/* One step of the layout: with `sealed` (device uint8[B], or NULL for none),
+ * every sequence whose open tail holds L tokens and whose sealed[b] is 0, 1
+ * or 2 has that chunk moved to segment sealed[b] (255: left open); then, with
+ * add_token = 1, one token row is reserved at the end of every sequence's
+ * open tail (a new tail is opened after a sealed chunk).  A layout that is
+ * not growable sets MQ_DEV_BAD_LAYOUT. */
+mq_status mq_grow_commit(const mq_shape* shape, void* layout, const uint8_t* sealed,
+                         int32_t add_token, void* stream);
+
+/* Writes the newest token of every sequence: K_new and V_new are device
+ * [B, Hkv, d] in kv_dtype (rows stored as fp16, round-to-nearest-even) into
+ * the row the last mq_grow_commit reserved in this layer's packed buffer.
+ * Sequences whose last commit found no room (MQ_GROW_FULL) are skipped. */
+mq_status mq_grow_append_kv(const mq_shape* shape, const void* layout,
+                            const void* K_new, const void* V_new, int32_t kv_dtype,
+                            void* packed, size_t packed_bytes, void* stream);
+
+/* Encodes every full open tail with sealed[b] in {1, 2} into the next free
+ * rows of that segment of this layer's packed buffer (the layout is not
+ * changed; the next mq_grow_commit with the same `sealed` moves the chunk). */
+mq_status mq_grow_seal(const mq_shape* shape, const void* layout, const uint8_t* sealed,
+                       void* packed, size_t packed_bytes, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

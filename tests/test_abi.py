@@ -167,3 +167,42 @@ def test_similarity_route_validation():
     many = np.full(70000, 1, np.int32)
     assert f(ctypes.byref(big), many.ctypes.data, p, p, 64, p, 0.1, 0.0, 1, p, None, 0) \
         == M.MQ_ERR_UNSUPPORTED
+
+
+def test_grow_sizes_and_validation():
+    shp = _shape(num_seqs=3, head_dim=128, chunk_len=64)
+    lens = np.array([300, 256, 0], np.int32)
+    lay, pk, ws = M.mq_grow_sizes(shp, lens, 100)
+    G = (100 + 63) // 64
+    n = (lens + 63) // 64
+    slots = int(n.sum()) + 3 * (G + 1)
+    pad16 = lambda x: (x + 15) // 16 * 16
+    assert lay == 64 + 3 * 160 + 2 * pad16(4 * slots)
+    # all present chunks at FP16 plus the reservations of the three segments
+    a128 = lambda x: (x + 127) // 128 * 128
+    want = 0
+    for nb in n.tolist():
+        want += 2 * 2 * (a128((nb + 1 + G) * 64 * 256)
+                         + a128(G * 64 * 64) + a128(G * 64 * 16)
+                         + a128(G * 64 * 32) + a128(G * 64 * 16))
+    assert pk == want
+    assert ws >= M.mq_decode_workspace_bytes(shp, lens)
+    lib = M.lib()
+    z = ctypes.c_size_t(0)
+    assert lib.mq_grow_sizes(ctypes.byref(shp), lens.ctypes.data, -1, ctypes.byref(z), None,
+                             None) == M.MQ_ERR_INVALID_ARG
+    big = np.array([1 << 23, 0, 0], np.int32)
+    assert lib.mq_grow_sizes(ctypes.byref(shp), big.ctypes.data, 1, ctypes.byref(z), None,
+                             None) == M.MQ_ERR_UNSUPPORTED
+    p = 1 << 20
+    assert lib.mq_grow_commit(ctypes.byref(shp), p, None, 2, 0) == M.MQ_ERR_INVALID_ARG
+    assert lib.mq_grow_commit(ctypes.byref(shp), p, p + 1, 1, 0) == M.MQ_ERR_INVALID_ARG
+    assert lib.mq_grow_seal(ctypes.byref(shp), p, None, p, 1 << 20, 0) == M.MQ_ERR_INVALID_ARG
+    assert lib.mq_grow_append_kv(ctypes.byref(shp), p, p, p, 5, p, 1 << 20, 0) \
+        == M.MQ_ERR_INVALID_ARG
+    need = lay
+    assert lib.mq_grow_build_layout(ctypes.byref(shp), lens.ctypes.data, 100, p, p, p, need - 16,
+                                    0) == M.MQ_ERR_WORKSPACE
+    # valid arguments, no device: a CUDA error, never a silent CPU path
+    assert lib.mq_grow_build_layout(ctypes.byref(shp), lens.ctypes.data, 100, p, p, p, need,
+                                    0) == M.MQ_ERR_CUDA
