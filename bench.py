@@ -56,6 +56,9 @@ def parse():
     p.add_argument("--lam", type=float, default=0.0,
                    help="memory-pressure knob for the router map: subtracts lam * bits/16 from "
                         "each expert's bias (more INT2 as lam grows, more FP16 below 0)")
+    p.add_argument("--grow", action="store_true",
+                   help="decode-time cache growth: every decode step appends one token per "
+                        "sequence; full tails are routed and sealed into their segments")
     p.add_argument("--no-rs", action="store_true",
                    help="routing sharing off: one router, map and layout per layer")
     return p.parse_args()
@@ -74,8 +77,8 @@ def measured_peaks():
 # workload, from an ncu capture (the command and counters are recorded under
 # profiles/), valid only for the pack sources with this SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "332f50ffc4a4f93ce6f1023404735377cbc393833f092325753fdb852f05c186",
-                "bytes_per_launch": 2154973952 + 856188416}
+                "sha256": "d0d0455b063152d6cab03b7dfb588d5755db3f95497c8a380df8cb9891443e49",
+                "bytes_per_launch": 2155172608 + 856218112}
 
 
 def pack_sources_sha256():
@@ -225,7 +228,8 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
 class Setup:
     """Device-resident inputs and outputs of one batch of the workload."""
 
-    def __init__(self, w, seed, device, routing_sharing=True, router="moqae", lam=0.0):
+    def __init__(self, w, seed, device, routing_sharing=True, router="moqae", lam=0.0,
+                 grow=False):
         import torch
         from chunk_adaptive_mixed_b200 import mqkv as M
         from chunk_adaptive_mixed_b200 import workloads as W
@@ -284,13 +288,114 @@ class Setup:
                                 device=device) for _ in range(w.layers)]
         self.ws = torch.empty(M.mq_decode_workspace_bytes(self.shape, self.lens), dtype=u8,
                               device=device)
+        self.grow = grow
+        if grow:
+            self._setup_grow(seed, device)
         self.kv_bytes = sum(K.numel() * K.element_size() * 2 for K in self.K) // w.layers
         torch.cuda.synchronize()
+
+    def _setup_grow(self, seed, device):
+        """Growable layout sized for decode_steps more tokens, the appended
+        tokens' K/V and router-input rows, and which sequences fill a chunk at
+        which step (lengths are known on the host)."""
+        import torch
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        from chunk_adaptive_mixed_b200 import workloads as W
+        w, u8 = self.w, torch.uint8
+        if self.router != "moqae" or not self.rs:
+            raise SystemExit("--grow runs with the MoQAE router and routing sharing")
+        n = w.decode_steps
+        lay_b, pk_b, ws_b = M.mq_grow_sizes(self.shape, self.lens, n)
+        self.cap_lens = self.lens + n
+        self.layouts = [torch.empty(lay_b, dtype=u8, device=device)]
+        self.layout = self.layouts[0]
+        self.packed = [torch.empty(pk_b, dtype=u8, device=device) for _ in range(w.layers)]
+        self.ws = torch.empty(ws_b, dtype=u8, device=device)
+        self.kv_new = [[W.new_token_kv(w, l, s, seed, device) for s in range(n)]
+                       for l in range(w.layers)]
+        self.c_new = [W.new_token_router_input(w, s, seed, device) for s in range(n)]
+        L, B = w.chunk_len, self.B
+        # router input of every sequence's open tail, [B * L, D]: the prefill's
+        # partial chunk, then one row per appended token
+        self.tail_c0 = torch.zeros(B * L, w.router_dim, dtype=torch.float32, device=device)
+        cu = W.cu_seqlens(self.lens)
+        for b in range(B):
+            t = int(self.lens[b]) % L
+            if t:
+                self.tail_c0[b * L:b * L + t] = self.C[int(cu[b + 1]) - t:int(cu[b + 1])]
+        self.tail_c = self.tail_c0.clone()
+        self.tail_lens = np.full(B, L, np.int32)
+        self.tail_cu = torch.as_tensor(W.cu_seqlens(self.tail_lens), device=device)
+        self.tail_te = torch.empty(B * L, dtype=u8, device=device)
+        self.tail_ce = torch.empty(max(B, 16), dtype=u8, device=device)
+        self.tail_ws = torch.empty(M.mq_route_workspace_bytes(self.shape, self.tail_lens,
+                                                              w.router_dim, w.router_hidden),
+                                   dtype=u8, device=device)
+        self.sealed = torch.full((max(B, 16),), 255, dtype=u8, device=device)
+        self.no_seal = torch.full((max(B, 16),), 255, dtype=u8, device=device)
+        self.tail_row, self.fill_mask, self.fills = [], [], []
+        lens = self.lens.astype(np.int64).copy()
+        for s in range(n):
+            pos = lens % L                          # row of the new token in its tail
+            self.tail_row.append(torch.as_tensor(np.arange(B) * L + pos, device=device))
+            lens += 1
+            full = lens % L == 0
+            mask = np.zeros(max(B, 16), bool)
+            mask[:B] = full
+            self.fill_mask.append(torch.as_tensor(mask, device=device))
+            self.fills.append(int(full.sum()))
+
+    def step_grow(self, timers=None):
+        """Prefill (route, growable layout, pack) then decode_steps decode
+        steps that each append one token per sequence before attending."""
+        import torch
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        w, n = self.w, self.w.decode_steps
+        if timers:
+            timers["route"][0].record()
+        M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, self.W1, self.W2, self.W3,
+                          self.b3, self.token_expert, self.chunk_expert, self.route_ws)
+        if timers:
+            timers["route"][1].record()
+        M.mq_grow_build_layout(self.shape, self.lens, n, self.cu, self.chunk_expert, self.layout)
+        for layer in range(w.layers):
+            if timers:
+                timers["pack"][layer][0].record()
+            M.mq_grow_pack_kv(self.shape, self.lens, n, self.layout, self.K[layer], self.V[layer],
+                              self.packed[layer])
+            if timers:
+                timers["pack"][layer][1].record()
+        self.tail_c.copy_(self.tail_c0)
+        pending = False
+        for s in range(n):
+            M.mq_grow_commit(self.shape, self.layout, self.sealed if pending else None, True)
+            self.tail_c.index_copy_(0, self.tail_row[s], self.c_new[s])
+            for layer in range(w.layers):
+                Kn, Vn = self.kv_new[layer][s]
+                M.mq_grow_append_kv(self.shape, self.layout, Kn, Vn, self.packed[layer])
+                if timers and s == 0:
+                    timers["decode"][layer][0].record()
+                M.mq_decode_attn(self.shape, self.cap_lens, self.layout, self.packed[layer],
+                                 self.q[layer][s], self.out[layer], self.ws)
+                if timers and s == 0:
+                    timers["decode"][layer][1].record()
+            pending = self.fills[s] > 0
+            if pending:
+                # route the full tails (all B tails are scored; only the full
+                # ones are sealed)
+                M.mq_route_chunks(self.shape, self.tail_lens, self.tail_cu, self.tail_c, self.W1,
+                                  self.W2, self.W3, self.b3, self.tail_te, self.tail_ce,
+                                  self.tail_ws, routing_freeze=False)
+                torch.where(self.fill_mask[s], self.tail_ce, self.no_seal, out=self.sealed)
+                for layer in range(w.layers):
+                    M.mq_grow_seal(self.shape, self.layout, self.sealed, self.packed[layer])
 
     def step(self, timers=None):
         """One pass of the whole path (launches only; asynchronous)."""
         from chunk_adaptive_mixed_b200 import mqkv as M
         w = self.w
+        if self.grow:
+            return self.step_grow(timers)
         if timers:
             timers["route"][0].record()
         for r, (W1, W2, W3, b3) in enumerate(self.routers):
@@ -325,6 +430,11 @@ class Setup:
         return self.layouts[0 if self.rs else layer]
 
     def launches_per_step(self):
+        if self.grow:
+            w, n = self.w, self.w.decode_steps
+            fill_steps = sum(1 for f in self.fills if f)
+            return (5 + w.layers + n * (2 + 3 * w.layers)
+                    + fill_steps * (3 + w.layers))
         # per map: weight split + router + vote (or one similarity kernel) and
         # 2 layout kernels; one pack per layer; two decode kernels per layer
         # and decode step
@@ -355,7 +465,8 @@ def run_ours(args, rank, world, local_rank):
     seed = rank_seed(args.seed, rank)
     if args.lam and args.router != "moqae":
         raise SystemExit("--lam applies to the MoQAE router only")
-    S = Setup(w, seed, device, routing_sharing=not args.no_rs, router=args.router, lam=args.lam)
+    S = Setup(w, seed, device, routing_sharing=not args.no_rs, router=args.router, lam=args.lam,
+              grow=args.grow)
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -368,7 +479,15 @@ def run_ours(args, rank, world, local_rank):
         S.step()
     torch.cuda.synchronize()
     assert M.mq_device_status() == 0, "device-side check failed during warm-up"
-    pb = int(np.mean([M.mq_packed_bytes(S.layout_of(l)) for l in range(w.layers)]))
+    if S.grow:
+        # bytes the prefill map occupies (a growable layout's header counts
+        # its reservations too): a fixed layout of the same map
+        fixed = torch.empty(M.mq_layout_bytes(S.shape, S.lens), dtype=torch.uint8, device=device)
+        M.mq_build_layout(S.shape, S.lens, S.cu, S.chunk_expert, fixed)
+        pb = M.mq_packed_bytes(fixed)
+        del fixed
+    else:
+        pb = int(np.mean([M.mq_packed_bytes(S.layout_of(l)) for l in range(w.layers)]))
     mix = np.bincount(S.chunk_expert[:S.N].cpu().numpy(), minlength=3) / max(S.N, 1)
 
     # per-kernel events for every pack launch and the first decode step
@@ -428,6 +547,7 @@ def run_ours(args, rank, world, local_rank):
                        "router_D": w.router_dim, "router_H": w.router_hidden,
                        "kv_dtype": w.kv_dtype, "decode_steps": w.decode_steps,
                        "routing_sharing": S.rs, "router": S.router, "lam": S.lam,
+                       "grow": bool(S.grow),
                        "parallelism": f"dp{world} (independent batches)",
                        "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
                        else "inputs fit in L2"},
@@ -470,8 +590,14 @@ def run_e2e(S, args, device):
     host["V"] = [pinned_copy(V) for V in S.V]
     host["q"] = [[pinned_copy(q) for q in qs] for qs in S.q]
     host["u"] = [pinned_copy(u) for u in S.u] if S.router == "similarity" else []
+    # decode-time growth: every appended token's K/V and router-input row
+    host["kv_new"] = ([[(pinned_copy(k), pinned_copy(v)) for k, v in per] for per in S.kv_new]
+                      if S.grow else [])
+    host["c_new"] = [pinned_copy(c) for c in S.c_new] if S.grow else []
     out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in S.out]
-    h2d = (host["C"].numel() * 4 + sum(u.numel() * 4 for u in host["u"]) + sum(x.numel() * x.element_size() for x in host["K"] + host["V"])
+    h2d = (host["C"].numel() * 4 + sum(u.numel() * 4 for u in host["u"])
+           + sum(k.numel() * k.element_size() * 2 for per in host["kv_new"] for k, _ in per)
+           + sum(c.numel() * 4 for c in host["c_new"]) + sum(x.numel() * x.element_size() for x in host["K"] + host["V"])
            + sum(q.numel() * q.element_size() for qs in host["q"] for q in qs))
     d2h = sum(o.numel() * o.element_size() for o in out_host) * w.decode_steps
 
@@ -479,6 +605,12 @@ def run_e2e(S, args, device):
         S.C.copy_(host["C"], non_blocking=True)
         for r, u in enumerate(host["u"]):
             S.u[r].copy_(u, non_blocking=True)
+        for layer, per in enumerate(host["kv_new"]):
+            for s_, (k, v) in enumerate(per):
+                S.kv_new[layer][s_][0].copy_(k, non_blocking=True)
+                S.kv_new[layer][s_][1].copy_(v, non_blocking=True)
+        for s_, c in enumerate(host["c_new"]):
+            S.c_new[s_].copy_(c, non_blocking=True)
         for layer in range(w.layers):
             S.K[layer].copy_(host["K"][layer], non_blocking=True)
             S.V[layer].copy_(host["V"][layer], non_blocking=True)

@@ -47,7 +47,7 @@ EXPERT_BITS = (16, 4, 2)
 
 # stream tags for seed derivation
 _TAG = {"seq_lens": 1, "c_chunk": 2, "c_token": 3, "w1": 4, "w2": 5, "w3": 6, "k": 7, "v": 8,
-        "q": 9, "outliers": 10, "map": 11, "u": 12}
+        "q": 9, "outliers": 10, "map": 11, "u": 12, "k_new": 13, "v_new": 14, "c_new": 15}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -273,6 +273,23 @@ def query(w: Workload, layer: int = 0, step: int = 0, seed: int = 0, device="cpu
     q = torch.randn(w.num_seqs, w.num_q_heads, w.head_dim,
                     generator=generator(device, seed + layer, _TAG["q"], step), device=device)
     return q.to(w.torch_dtype)
+
+
+def new_token_kv(w: Workload, layer: int = 0, step: int = 0, seed: int = 0, device="cpu"):
+    """K, V [B, Hkv, d] of the token each sequence appends at decode step
+    `step` (a fresh draw per (layer, step), the workload's dtype)."""
+    shape = (w.num_seqs, w.num_kv_heads, w.head_dim)
+    K = torch.randn(*shape, generator=generator(device, seed + layer, _TAG["k_new"], step),
+                    device=device)
+    V = torch.randn(*shape, generator=generator(device, seed + layer, _TAG["v_new"], step),
+                    device=device)
+    return K.to(w.torch_dtype), V.to(w.torch_dtype)
+
+
+def new_token_router_input(w: Workload, step: int = 0, seed: int = 0, device="cpu"):
+    """Router input rows [B, D] fp32 of the tokens appended at decode step `step`."""
+    return torch.randn(w.num_seqs, w.router_dim,
+                       generator=generator(device, seed, _TAG["c_new"], step), device=device)
 
 
 def synthetic_chunk_map(lens: np.ndarray, chunk_len: int, mix=(0.2, 0.5, 0.3), seed: int = 0,
