@@ -563,9 +563,13 @@ static void decode_row(const uint8_t* region, uint64_t scale_off, int d, int e, 
  *   score_t = scale * <q, k_t>,  o = sum_t exp(score_t - max) v_t / sum_t exp(score_t - max)
  * K, V are n rows of d doubles.  n == 0 gives zeros.
  */
-static void attend(int n, int d, const double* q, const double* Kd, const double* Vd, double scale,
-                   double* o) {
+static void attend_ml(int n, int d, const double* q, const double* Kd, const double* Vd,
+                      double scale, double* o, double* ml) {
   for (int j = 0; j < d; ++j) o[j] = 0.0;
+  if (ml) {
+    ml[0] = -INFINITY;
+    ml[1] = 0.0;
+  }
   if (n == 0) return;
   double* sc = (double*)malloc(sizeof(double) * (size_t)n);
   double mx = -INFINITY;
@@ -582,7 +586,16 @@ static void attend(int n, int d, const double* q, const double* Kd, const double
     for (int j = 0; j < d; ++j) o[j] += p * Vd[(int64_t)t * d + j];
   }
   for (int j = 0; j < d; ++j) o[j] /= den;
+  if (ml) {
+    ml[0] = mx;   /* largest scaled score */
+    ml[1] = den;  /* sum of exp(score - mx) */
+  }
   free(sc);
+}
+
+static void attend(int n, int d, const double* q, const double* Kd, const double* Vd, double scale,
+                   double* o) {
+  attend_ml(n, d, q, Kd, Vd, scale, o, 0);
 }
 
 /*
@@ -591,9 +604,9 @@ static void attend(int n, int d, const double* q, const double* Kd, const double
  * g = h / (Hq/Hkv).  q is [B, Hq, d] (dtype 0 fp32, 1 fp16); scale <= 0 means
  * 1/sqrt(d).  out is [B, Hq, d] fp64.
  */
-void mqo_decode(int B, int Hq, int Hkv, int d, int L, const int32_t* seq_lens,
-                const uint8_t* chunk_expert, const uint8_t* packed, const void* q, int q_dtype,
-                double scale, double* out) {
+static void decode_impl(int B, int Hq, int Hkv, int d, int L, const int32_t* seq_lens,
+                        const uint8_t* chunk_expert, const uint8_t* packed, const void* q,
+                        int q_dtype, double scale, double* out, double* ml) {
   if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
   const int64_t N = mqo_num_chunks(B, seq_lens, L);
   int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * (size_t)(N > 0 ? N : 1));
@@ -630,13 +643,31 @@ void mqo_decode(int B, int Hq, int Hkv, int d, int L, const int32_t* seq_lens,
       decode_row(rk, s->scale_offset[e], d, e, segrow, Kd + (int64_t)t * d);
       decode_row(rv, s->scale_offset[e], d, e, segrow, Vd + (int64_t)t * d);
     }
-    attend(Tb, d, qd, Kd, Vd, scale, out + bh * d);
+    attend_ml(Tb, d, qd, Kd, Vd, scale, out + bh * d, ml ? ml + 2 * bh : 0);
     free(Kd);
     free(Vd);
   }
   free(perm);
   free(inv);
   free(si);
+}
+
+void mqo_decode(int B, int Hq, int Hkv, int d, int L, const int32_t* seq_lens,
+                const uint8_t* chunk_expert, const uint8_t* packed, const void* q, int q_dtype,
+                double scale, double* out) {
+  decode_impl(B, Hq, Hkv, d, L, seq_lens, chunk_expert, packed, q, q_dtype, scale, out, 0);
+}
+
+/*
+ * The same attention, also returning for every (b, h) the largest scaled
+ * score m and l = sum_t exp(score_t - m) (ml is [B, Hq, 2] fp64; an empty
+ * sequence gives m = -inf, l = 0).  These are what a device holding only part
+ * of a sequence's context contributes to the merge of a split softmax.
+ */
+void mqo_decode_partial(int B, int Hq, int Hkv, int d, int L, const int32_t* seq_lens,
+                        const uint8_t* chunk_expert, const uint8_t* packed, const void* q,
+                        int q_dtype, double scale, double* out, double* ml) {
+  decode_impl(B, Hq, Hkv, d, L, seq_lens, chunk_expert, packed, q, q_dtype, scale, out, ml);
 }
 
 /*

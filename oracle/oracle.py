@@ -64,6 +64,9 @@ def lib():
         L.mqo_dense_attention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           _i32p, _vp, _vp, ctypes.c_int, _vp, ctypes.c_int,
                                           ctypes.c_double, _f64p]
+        L.mqo_decode_partial.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, _i32p, _u8p, _u8p, _vp, ctypes.c_int,
+                                         ctypes.c_double, _f64p, _f64p]
         L.mqo_similarity_route.argtypes = [ctypes.c_int, _i32p, ctypes.c_int, ctypes.c_int, _f32p,
                                            _f32p, ctypes.c_double, ctypes.c_double, ctypes.c_int,
                                            _u8p, _f64p]
@@ -257,6 +260,21 @@ def decode(Hq, Hkv, d, L, seq_lens, chunk_expert, packed, q, scale=0.0):
                      _p(out, _f64p))
     return out
 
+
+
+def decode_partial(Hq, Hkv, d, L, seq_lens, chunk_expert, packed, q, scale=0.0):
+    """decode plus (m, l) per (b, h): out [B, Hq, d], ml [B, Hq, 2] (fp64)."""
+    sl = _c(seq_lens, np.int32)
+    ce = _c(chunk_expert, np.uint8)
+    packed = _c(packed, np.uint8)
+    q = np.ascontiguousarray(q)
+    B = len(sl)
+    out = np.empty((B, Hq, d), np.float64)
+    ml = np.empty((B, Hq, 2), np.float64)
+    lib().mqo_decode_partial(B, int(Hq), int(Hkv), int(d), int(L), _p(sl, _i32p), _p(ce, _u8p),
+                             _p(packed, _u8p), q.ctypes.data, _dtype_code(q), float(scale),
+                             _p(out, _f64p), _p(ml, _f64p))
+    return out, ml
 
 def decode_pairs(Hq, Hkv, d, L, seq_lens, chunk_expert, K, V, q, pairs, scale=0.0):
     """fp64 attention for selected (b, h) pairs from raw K/V; out [n, d]."""

@@ -576,3 +576,55 @@ def test_similarity_route_tail_zero_and_freeze():
     assert ce.tolist() == [2, 2, 2]
     ce, _ = O.similarity_route(lens, L, C, u, tau_hi=0.5, tau_lo=0.25, routing_freeze=True)
     assert ce.tolist() == [0, 2, 0]
+
+
+# ------------------------------------------------------ context-split records
+
+def test_decode_partial_two_token_closed_form():
+    # K rows a multiple of e0, q = 2 e0: scores scale * 2 * x_t; all FP16, exact in fp16
+    d, L = 64, 32
+    K = np.zeros((2, 1, d), np.float32)
+    V = np.zeros((2, 1, d), np.float32)
+    K[0, 0, 0], K[1, 0, 0] = 1.5, -0.75
+    V[0, 0, 1], V[1, 0, 2] = 1.0, 1.0
+    q = np.zeros((1, 1, d), np.float32)
+    q[0, 0, 0] = 2.0
+    lens = np.array([2], np.int32)
+    ce = np.zeros(1, np.uint8)
+    ref = O.pack(1, d, L, lens, ce, K, V)
+    o, ml = O.decode_partial(1, 1, d, L, lens, ce, ref, q)
+    s = np.array([3.0, -1.5]) / np.sqrt(d)
+    assert abs(ml[0, 0, 0] - s[0]) < 1e-15
+    assert abs(ml[0, 0, 1] - (1.0 + np.exp(s[1] - s[0]))) < 1e-15
+    p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+    assert np.allclose(o[0, 0, 1:3], p, atol=1e-15)
+
+
+def test_decode_partial_records_merge_to_the_whole_sequence():
+    # a sequence cut at a chunk boundary: the two shards' records, merged with
+    # the split-softmax rule, give the attention over the whole sequence
+    rng = np.random.default_rng(5)
+    d, L, Hkv, Hq = 64, 32, 2, 4
+    T, cut = 5 * L - 7, 2 * L
+    K = (rng.standard_normal((T, Hkv, d)) * 1.3).astype(np.float32)
+    V = rng.standard_normal((T, Hkv, d)).astype(np.float32)
+    q = rng.standard_normal((1, Hq, d)).astype(np.float32)
+    cmap = np.array([0, 2, 1, 1, 2], np.uint8)
+    full = np.array([T], np.int32)
+    ref = O.pack(Hkv, d, L, full, cmap, K, V)
+    o_full, ml_full = O.decode_partial(Hq, Hkv, d, L, full, cmap, ref, q)
+    recs = []
+    for lo, hi, m in [(0, cut, cmap[:2]), (cut, T, cmap[2:])]:
+        lens = np.array([hi - lo], np.int32)
+        r = O.pack(Hkv, d, L, lens, m, K[lo:hi], V[lo:hi])
+        recs.append(O.decode_partial(Hq, Hkv, d, L, lens, m, r, q))
+    M = np.maximum(recs[0][1][..., 0], recs[1][1][..., 0])
+    w = [ml[..., 1] * np.exp(ml[..., 0] - M) for _, ml in recs]
+    merged = (w[0][..., None] * recs[0][0] + w[1][..., None] * recs[1][0]) / (w[0] + w[1])[..., None]
+    assert np.allclose(merged, o_full, rtol=0, atol=1e-12)
+    assert np.allclose(M, ml_full[..., 0], atol=1e-14)
+    assert np.allclose(w[0] + w[1], ml_full[..., 1], rtol=1e-12)
+    # an empty shard contributes nothing
+    z = O.decode_partial(Hq, Hkv, d, L, np.array([0], np.int32), np.zeros(0, np.uint8),
+                         np.zeros(16, np.uint8), q)
+    assert np.all(z[1][..., 0] == -np.inf) and np.all(z[1][..., 1] == 0) and np.all(z[0] == 0)
