@@ -56,6 +56,9 @@ def parse():
     p.add_argument("--lam", type=float, default=0.0,
                    help="memory-pressure knob for the router map: subtracts lam * bits/16 from "
                         "each expert's bias (more INT2 as lam grows, more FP16 below 0)")
+    p.add_argument("--context-split", action="store_true",
+                   help="every rank holds a contiguous range of chunks of the same batch; "
+                        "per-rank partial records are all-gathered and merged (strong scaling)")
     p.add_argument("--grow", action="store_true",
                    help="decode-time cache growth: every decode step appends one token per "
                         "sequence; full tails are routed and sealed into their segments")
@@ -75,16 +78,17 @@ def measured_peaks():
 
 # DRAM bytes (read + write) of one full-size pack launch of the default
 # workload, from an ncu capture (the command and counters are recorded under
-# profiles/), valid only for the pack sources with this SHA-256.
+# profiles/), valid only for the pack kernel source (pack.cu) with this
+# SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "d0d0455b063152d6cab03b7dfb588d5755db3f95497c8a380df8cb9891443e49",
+                "sha256": "7742da4223f6323a87c63055c1133fcdf114037ed7413ea3c5cf0283c07bb5e3",
                 "bytes_per_launch": 2155172608 + 856218112}
 
 
 def pack_sources_sha256():
     import hashlib
     h = hashlib.sha256()
-    for f in ("pack.cu", "common.cuh"):
+    for f in ("pack.cu",):
         with open(os.path.join(ROOT, "chunk_adaptive_mixed_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -229,12 +233,24 @@ class Setup:
     """Device-resident inputs and outputs of one batch of the workload."""
 
     def __init__(self, w, seed, device, routing_sharing=True, router="moqae", lam=0.0,
-                 grow=False):
+                 grow=False, shard=None):
         import torch
+        from chunk_adaptive_mixed_b200 import context_split as CS
         from chunk_adaptive_mixed_b200 import mqkv as M
         from chunk_adaptive_mixed_b200 import workloads as W
         self.w = w
-        self.lens = W.seq_lens(w, seed)
+        # shard = (rank, world): this rank holds a contiguous range of whole
+        # chunks of every sequence of one shared batch (context split)
+        self.shard = shard
+        self.full_lens = W.seq_lens(w, seed)
+        if shard is not None:
+            rank, world = shard
+            self.lo, self.hi = CS.shard_ranges(self.full_lens, w.chunk_len, rank, world)
+            self.lens = CS.shard_lengths(self.full_lens, w.chunk_len, rank, world)
+            self.freeze = CS.routing_freeze(rank)
+        else:
+            self.lens = self.full_lens
+            self.freeze = True
         self.B = len(self.lens)
         self.T = int(self.lens.sum())
         self.N = int(W.num_chunks(self.lens, w.chunk_len).sum())
@@ -262,12 +278,15 @@ class Setup:
             self.u = [W.similarity_query(w, seed + (l if not routing_sharing else 0), device)
                       for l in range(nr)]
             self.tau = W.similarity_thresholds(w)
-        self.C = W.router_input(w, self.lens, seed, device)
+        take = (lambda x: CS.shard_rows(x, self.full_lens, self.lo, self.hi)) if shard else \
+            (lambda x: x)
+        self.C = take(W.router_input(w, self.full_lens, seed, device))
         self.K, self.V, self.q = [], [], []
         for layer in range(w.layers):
-            K, V = W.kv_layer(w, self.lens, layer, seed, device)
-            self.K.append(K)
-            self.V.append(V)
+            K, V = W.kv_layer(w, self.full_lens, layer, seed, device)
+            self.K.append(take(K))
+            self.V.append(take(V))
+            del K, V
             self.q.append([W.query(w, layer, s, seed, device) for s in range(w.decode_steps)])
         u8 = torch.uint8
         self.route_ws = torch.empty(M.mq_route_workspace_bytes(self.shape, self.lens, w.router_dim,
@@ -280,17 +299,29 @@ class Setup:
                                     device=device) for _ in range(nr)]
         self.chunk_expert = self.chunk_experts[0]
         self.layout = self.layouts[0]
-        # packed buffers sized for any routing map (all-FP16 bound): no host
-        # round trip is needed between routing and packing
-        ub = M.mq_packed_bytes_upper_bound(self.shape, self.lens)
-        self.packed = [torch.empty(ub, dtype=u8, device=device) for _ in range(w.layers)]
+        # packed buffers: the inputs are the same every step, so the map is
+        # too; route once here and size every buffer at the packed bytes of
+        # its layout (no host round trip separates routing from packing in
+        # the timed steps; a larger map would be caught by the pack kernel's
+        # capacity check)
+        self._route_maps()
+        self._build_layouts()
+        need = max(M.mq_packed_bytes(lay) for lay in self.layouts)
+        self.packed = [torch.empty(max(need, 16), dtype=u8, device=device)
+                       for _ in range(w.layers)]
         self.out = [torch.empty(self.B, w.num_q_heads, w.head_dim, dtype=torch.float32,
                                 device=device) for _ in range(w.layers)]
         self.ws = torch.empty(M.mq_decode_workspace_bytes(self.shape, self.lens), dtype=u8,
                               device=device)
         self.grow = grow
         if grow:
+            if shard is not None:
+                raise SystemExit("--grow and --context-split are separate variants")
             self._setup_grow(seed, device)
+        if shard is not None:
+            # this rank's records, all ranks' records, the merged output
+            d4 = M.partial_floats(w.head_dim)
+            self.rec = torch.empty(self.B, w.num_q_heads, d4, dtype=torch.float32, device=device)
         self.kv_bytes = sum(K.numel() * K.element_size() * 2 for K in self.K) // w.layers
         torch.cuda.synchronize()
 
@@ -398,18 +429,10 @@ class Setup:
             return self.step_grow(timers)
         if timers:
             timers["route"][0].record()
-        for r, (W1, W2, W3, b3) in enumerate(self.routers):
-            if self.router == "similarity":
-                M.mq_similarity_route(self.shape, self.lens, self.cu, self.C, self.u[r],
-                                      self.tau[0], self.tau[1], self.chunk_experts[r])
-            else:
-                M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, W1, W2, W3, b3,
-                                  self.token_expert, self.chunk_experts[r], self.route_ws)
+        self._route_maps()
         if timers:
             timers["route"][1].record()
-        for r in range(len(self.routers)):
-            M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_experts[r],
-                              self.layouts[r])
+        self._build_layouts()
         for layer in range(w.layers):
             if timers:
                 timers["pack"][layer][0].record()
@@ -421,15 +444,47 @@ class Setup:
             for layer in range(w.layers):
                 if timers and s == 0:
                     timers["decode"][layer][0].record()
-                M.mq_decode_attn(self.shape, self.lens, self.layout_of(layer),
-                                 self.packed[layer], self.q[layer][s], self.out[layer], self.ws)
+                if self.shard is None:
+                    M.mq_decode_attn(self.shape, self.lens, self.layout_of(layer),
+                                     self.packed[layer], self.q[layer][s], self.out[layer],
+                                     self.ws)
+                else:
+                    self.decode_split(layer, s)
                 if timers and s == 0:
                     timers["decode"][layer][1].record()
+
+    def _route_maps(self):
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        for r, (W1, W2, W3, b3) in enumerate(self.routers):
+            if self.router == "similarity":
+                M.mq_similarity_route(self.shape, self.lens, self.cu, self.C, self.u[r],
+                                      self.tau[0], self.tau[1], self.chunk_experts[r])
+            else:
+                M.mq_route_chunks(self.shape, self.lens, self.cu, self.C, W1, W2, W3, b3,
+                                  self.token_expert, self.chunk_experts[r], self.route_ws,
+                                  routing_freeze=self.freeze)
+
+    def _build_layouts(self):
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        for r in range(len(self.routers)):
+            M.mq_build_layout(self.shape, self.lens, self.cu, self.chunk_experts[r],
+                              self.layouts[r])
+
+    def decode_split(self, layer, s):
+        """This rank's records, the all-gather over every rank, the merge."""
+        from chunk_adaptive_mixed_b200 import context_split as CS
+        from chunk_adaptive_mixed_b200 import mqkv as M
+        M.mq_decode_attn_partial(self.shape, self.lens, self.layout_of(layer), self.packed[layer],
+                                 self.q[layer][s], self.rec, self.ws)
+        M.mq_combine_partials(CS.gather_records(self.rec), self.out[layer])
 
     def layout_of(self, layer):
         return self.layouts[0 if self.rs else layer]
 
     def launches_per_step(self):
+        if self.shard is not None:   # partial decode (2) + combine (1) per layer and step
+            return (5 * len(self.routers) + self.w.layers
+                    + 3 * self.w.layers * self.w.decode_steps)
         if self.grow:
             w, n = self.w, self.w.decode_steps
             fill_steps = sum(1 for f in self.fills if f)
@@ -462,11 +517,13 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     w = workload(args)
-    seed = rank_seed(args.seed, rank)
+    # independent batches per rank (weak scaling), or one shared batch split
+    # by context (strong scaling)
+    seed = args.seed if args.context_split else rank_seed(args.seed, rank)
     if args.lam and args.router != "moqae":
         raise SystemExit("--lam applies to the MoQAE router only")
     S = Setup(w, seed, device, routing_sharing=not args.no_rs, router=args.router, lam=args.lam,
-              grow=args.grow)
+              grow=args.grow, shard=(rank, world) if args.context_split else None)
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -519,7 +576,10 @@ def run_ours(args, rank, world, local_rank):
     dec_avg = float(np.mean(dec_ms))
 
     tokens_per_step = S.B * w.decode_steps
-    value = job_throughput(tokens_per_step, world, ms_step)
+    if args.context_split:
+        value = tokens_per_step / (ms_step / 1e3)    # every rank works on the same sequences
+    else:
+        value = job_throughput(tokens_per_step, world, ms_step)
     peak, peak_kind = measured_peaks()
     pack_bytes = S.kv_bytes + pb                                   # read K/V, write packed
     dec_bytes = pb + sum(x.numel() * x.element_size() for x in (S.q[0][0], S.out[0]))
@@ -538,17 +598,20 @@ def run_ours(args, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "strong" if args.context_split else "weak",
+            "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded; random tensors of the model's shape, no checkpoint)",
             "config": {"workload": w.name, "layers": w.layers, "num_seqs": S.B,
-                       "seq_len": int(S.lens.max()), "total_tokens": S.T,
+                       "seq_len": int(S.full_lens.max()), "total_tokens": int(S.full_lens.sum()),
                        "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
                        "head_dim": w.head_dim, "chunk_len": w.chunk_len,
                        "router_D": w.router_dim, "router_H": w.router_hidden,
                        "kv_dtype": w.kv_dtype, "decode_steps": w.decode_steps,
                        "routing_sharing": S.rs, "router": S.router, "lam": S.lam,
                        "grow": bool(S.grow),
-                       "parallelism": f"dp{world} (independent batches)",
+                       "parallelism": (f"cp{world} (context split, records all-gathered)"
+                                       if args.context_split
+                                       else f"dp{world} (independent batches)"),
                        "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
                        else "inputs fit in L2"},
             "roofline": {"bound": "hbm", "kernel": "pack_kernel",

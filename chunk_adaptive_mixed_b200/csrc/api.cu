@@ -430,6 +430,52 @@ mq_status mq_decode_attn(const mq_shape* shape, const int32_t* h_seq_lens, const
   return MQ_OK;
 }
 
+// ------------------------------------------------------------ context split
+
+mq_status mq_decode_attn_partial(const mq_shape* shape, const int32_t* h_seq_lens,
+                                 const void* layout, const void* packed, const void* q,
+                                 int32_t q_dtype, float softmax_scale, float* partial,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  MQ_TRY(check_shape(shape));
+  int64_t T, N;
+  MQ_TRY(check_lens(shape, h_seq_lens, &T, &N));
+  if (q_dtype != MQ_F16 && q_dtype != MQ_F32)
+    return fail(MQ_ERR_INVALID_ARG, "q_dtype must be MQ_F16 or MQ_F32 (got %d)", q_dtype);
+  MQ_NEED_PTR(layout, "layout");
+  MQ_NEED_PTR(q, "q");
+  MQ_NEED_PTR(partial, "partial");
+  if (T > 0) MQ_NEED_PTR(packed, "packed");
+  const ItemPolicy p = item_policy(*shape, h_seq_lens);
+  const int64_t items = max_items_per_kv_head(*shape, h_seq_lens, p);
+  const size_t need = decode_workspace_bytes(*shape, items);
+  if (workspace_bytes < need)
+    return fail(MQ_ERR_WORKSPACE, "workspace_bytes %zu < %zu needed", workspace_bytes, need);
+  MQ_NEED_PTR(workspace, "workspace");
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / sqrtf((float)shape->head_dim);
+  unsigned int* status = nullptr;
+  cudaError_t err = status_word(&status);
+  if (err != cudaSuccess) return cuda_fail(err, "device status word");
+  err = launch_decode(*shape, items, layout, packed, q, q_dtype, softmax_scale, partial, workspace,
+                      workspace_bytes, status, static_cast<cudaStream_t>(stream), true);
+  if (err != cudaSuccess) return cuda_fail(err, "decode launch");
+  return MQ_OK;
+}
+
+mq_status mq_combine_partials(int32_t num_parts, int32_t num_seqs, int32_t num_q_heads,
+                              int32_t head_dim, const float* partials, float* out, void* stream) {
+  if (num_parts < 1) return fail(MQ_ERR_INVALID_ARG, "num_parts must be >= 1 (got %d)", num_parts);
+  if (num_seqs < 1 || num_q_heads < 1)
+    return fail(MQ_ERR_INVALID_ARG, "num_seqs and num_q_heads must be >= 1");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(MQ_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  MQ_NEED_PTR(partials, "partials");
+  MQ_NEED_PTR(out, "out");
+  const cudaError_t err = launch_combine_partials(num_parts, num_seqs, num_q_heads, head_dim,
+                                                  partials, out, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "combine launch");
+  return MQ_OK;
+}
+
 // ---------------------------------------------------------------- growth
 
 mq_status mq_grow_sizes(const mq_shape* shape, const int32_t* h_seq_lens, int32_t grow_tokens,

@@ -136,10 +136,13 @@ cudaError_t launch_grow_append(const mq_shape& s, const void* layout, const void
 cudaError_t launch_pack(const mq_shape& s, int64_t total_chunks, const void* layout, const void* K,
                         const void* V, int kv_dtype, void* packed, uint64_t packed_bytes,
                         unsigned int* status, cudaStream_t stream);
+// partial: write context-shard records [B, Hq, d + 4] instead of the output.
 cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layout,
                           const void* packed, const void* q, int q_dtype, float softmax_scale,
                           float* out, void* workspace, size_t workspace_bytes,
-                          unsigned int* status, cudaStream_t stream);
+                          unsigned int* status, cudaStream_t stream, bool partial = false);
+cudaError_t launch_combine_partials(int P, int B, int Hq, int D, const float* parts, float* out,
+                                    cudaStream_t stream);
 
 // Records a formatted reason for mq_last_error() and returns `status`.
 mq_status report_error(mq_status status, const char* fmt, ...);

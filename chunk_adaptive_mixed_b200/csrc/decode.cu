@@ -516,7 +516,11 @@ decode_partial_kernel(const unsigned char* __restrict__ layout,
 // One CTA per (sequence, query head): 8 warps split the items, each keeps a
 // running (max, sum, accumulator) over its items, then the warps' states are
 // merged in shared memory.
-template <int D, int QPG>
+// PARTIAL: instead of the attention output, write the record of a context
+// shard: [o (D values, normalised), m, l, 0, 0] with m the reference score of
+// the merged softmax (natural-log units, within 8 ln 2 below the largest
+// score) and l = sum exp(score - m) (mq_decode_attn_partial).
+template <int D, int QPG, bool PARTIAL>
 __global__ void __launch_bounds__(256)
 decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
                       const float* __restrict__ ws_acc, const float2* __restrict__ ws_ml,
@@ -575,15 +579,54 @@ decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
       num += f * s_acc[w][threadIdx.x];
       den += f * s_l[w];
     }
-    out[bh * D + threadIdx.x] = den > 0.f ? num / den : 0.f;
+    if constexpr (PARTIAL) {
+      float* rec = out + bh * (D + 4);
+      rec[threadIdx.x] = den > 0.f ? num / den : 0.f;
+      if (threadIdx.x == 0) {
+        rec[D] = den > 0.f ? Mx * 0.6931471805599453f : -INFINITY;  // log2 -> natural units
+        rec[D + 1] = den;
+        rec[D + 2] = 0.f;
+        rec[D + 3] = 0.f;
+      }
+    } else {
+      out[bh * D + threadIdx.x] = den > 0.f ? num / den : 0.f;
+    }
   }
+}
+
+// Merge of P context-shard records per (sequence, query head):
+//   M = max_r m_r,  w_r = l_r exp(m_r - M),  o = sum_r w_r o_r / sum_r w_r
+// (0 when every shard is empty).  One CTA per (b, h), one thread per value.
+__global__ void __launch_bounds__(128)
+combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ parts,
+                        float* __restrict__ out) {
+  const int64_t bh = blockIdx.x;
+  const int i = threadIdx.x;
+  if (i >= D) return;  // no barrier below
+  const size_t rec = (size_t)D + 4;
+  float M = -INFINITY;
+  for (int r = 0; r < P; ++r) {
+    const float* p = parts + ((size_t)r * heads + bh) * rec;
+    if (p[D + 1] > 0.f) M = fmaxf(M, p[D]);
+  }
+  float num = 0.f, den = 0.f;
+  for (int r = 0; r < P; ++r) {
+    const float* p = parts + ((size_t)r * heads + bh) * rec;
+    const float l = p[D + 1];
+    if (l > 0.f) {
+      const float w = l * expf(p[D] - M);
+      num = fmaf(w, p[i], num);
+      den += w;
+    }
+  }
+  out[bh * D + i] = den > 0.f ? num / den : 0.f;
 }
 
 template <int D, int QPG, int QDT>
 cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layout,
                             const unsigned char* packed, const void* q, float scale_log2,
                             float* out, float* ws_acc, float2* ws_ml, int num_seqs,
-                            unsigned int* status, cudaStream_t stream) {
+                            unsigned int* status, cudaStream_t stream, bool partial) {
   constexpr size_t smem = decode_smem_bytes<D, QPG>();
   auto kern = decode_partial_kernel<D, QPG, QDT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -603,7 +646,12 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   const int64_t heads = (int64_t)num_seqs * Hq;
-  decode_combine_kernel<D, QPG><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc, ws_ml, out);
+  if (partial)
+    decode_combine_kernel<D, QPG, true><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc,
+                                                                             ws_ml, out);
+  else
+    decode_combine_kernel<D, QPG, false><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc,
+                                                                              ws_ml, out);
   return cudaGetLastError();
 }
 
@@ -611,12 +659,12 @@ template <int D, int QDT>
 cudaError_t dispatch_qpg(int qpg, int64_t max_items, int Hq, const unsigned char* layout,
                          const unsigned char* packed, const void* q, float scale_log2, float* out,
                          float* ws_acc, float2* ws_ml, int B, unsigned int* status,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, bool partial) {
   switch (qpg) {
-    case 1: return launch_decode_t<D, 1, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream);
-    case 2: return launch_decode_t<D, 2, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream);
-    case 4: return launch_decode_t<D, 4, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream);
-    case 8: return launch_decode_t<D, 8, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream);
+    case 1: return launch_decode_t<D, 1, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
+    case 2: return launch_decode_t<D, 2, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
+    case 4: return launch_decode_t<D, 4, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
+    case 8: return launch_decode_t<D, 8, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -632,7 +680,7 @@ size_t decode_workspace_bytes(const mq_shape& s, int64_t max_items) {
 cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layout,
                           const void* packed, const void* q, int q_dtype, float softmax_scale,
                           float* out, void* workspace, size_t workspace_bytes,
-                          unsigned int* status, cudaStream_t stream) {
+                          unsigned int* status, cudaStream_t stream, bool partial) {
   (void)workspace_bytes;
   const int64_t qpg = s.num_q_heads / s.num_kv_heads;
   const int64_t recs = max_items * s.num_kv_heads * qpg;
@@ -645,12 +693,20 @@ cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layo
   const int64_t cap = max_items * s.num_kv_heads;
   if (s.head_dim == 128) {
     if (q_dtype == MQ_F16)
-      return dispatch_qpg<128, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream);
-    return dispatch_qpg<128, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream);
+      return dispatch_qpg<128, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
+    return dispatch_qpg<128, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
   }
   if (q_dtype == MQ_F16)
-    return dispatch_qpg<64, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream);
-  return dispatch_qpg<64, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream);
+    return dispatch_qpg<64, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
+  return dispatch_qpg<64, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
+}
+
+cudaError_t launch_combine_partials(int P, int B, int Hq, int D, const float* parts, float* out,
+                                    cudaStream_t stream) {
+  const int64_t heads = (int64_t)B * Hq;
+  if (heads == 0) return cudaSuccess;
+  combine_partials_kernel<<<(unsigned)heads, 128, 0, stream>>>(P, heads, D, parts, out);
+  return cudaGetLastError();
 }
 
 }  // namespace mqkv

@@ -41,7 +41,7 @@ EXPORTS = ("mq_status_string", "mq_last_error", "mq_layout_bytes", "mq_packed_by
            "mq_decode_workspace_bytes", "mq_route_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
            "mq_similarity_route", "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc",
            "mq_grow_sizes", "mq_grow_build_layout", "mq_grow_pack_kv", "mq_grow_commit",
-           "mq_grow_append_kv", "mq_grow_seal")
+           "mq_grow_append_kv", "mq_grow_seal", "mq_decode_attn_partial", "mq_combine_partials")
 
 # size of the scratch array built into the library for mq_decode_attn_noalloc
 MQ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -112,6 +112,10 @@ def lib() -> ctypes.CDLL:
     L.mq_grow_append_kv.argtypes = [sp, vp, vp, vp, i32, vp, sz, vp]
     L.mq_grow_seal.restype = ctypes.c_int
     L.mq_grow_seal.argtypes = [sp, vp, vp, vp, sz, vp]
+    L.mq_decode_attn_partial.restype = ctypes.c_int
+    L.mq_decode_attn_partial.argtypes = [sp, vp, vp, vp, vp, i32, ctypes.c_float, vp, vp, sz, vp]
+    L.mq_combine_partials.restype = ctypes.c_int
+    L.mq_combine_partials.argtypes = [i32, i32, i32, i32, vp, vp, vp]
     L.mq_pack_kv.restype = ctypes.c_int
     L.mq_pack_kv.argtypes = [sp, vp, vp, vp, vp, i32, vp, sz, vp]
     L.mq_decode_attn.restype = ctypes.c_int
@@ -316,3 +320,27 @@ def mq_grow_seal(shp, layout, sealed, packed, stream=None):
     nbytes = packed.numel() * packed.element_size()
     _check(lib().mq_grow_seal(ctypes.byref(shp), _ptr(layout), _ptr(sealed), _ptr(packed), nbytes,
                               _stream(stream)), "mq_grow_seal")
+
+
+# ------------------------------------------------------------ context split
+
+def partial_floats(head_dim: int) -> int:
+    """Floats of one (sequence, head) record of mq_decode_attn_partial."""
+    return head_dim + 4
+
+
+def mq_decode_attn_partial(shp, seq_lens, layout, packed, q, partial, workspace,
+                           softmax_scale=0.0, stream=None):
+    l = _lens(seq_lens)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().mq_decode_attn_partial(ctypes.byref(shp), l.ctypes.data, _ptr(layout),
+                                        _ptr(packed), _ptr(q), _dtype_code(q),
+                                        float(softmax_scale), _ptr(partial), _ptr(workspace),
+                                        nbytes, _stream(stream)), "mq_decode_attn_partial")
+
+
+def mq_combine_partials(partials, out, stream=None):
+    """partials [P, B, Hq, d + 4] fp32 -> out [B, Hq, d] fp32."""
+    P, B, Hq, rec = partials.shape
+    _check(lib().mq_combine_partials(int(P), int(B), int(Hq), int(rec - 4), _ptr(partials),
+                                     _ptr(out), _stream(stream)), "mq_combine_partials")

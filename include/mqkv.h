@@ -22,6 +22,9 @@
  *                    from the mixed-bitwidth packed cache.
  *   mq_grow_*        decode-time growth: new tokens in an FP16 tail, each full
  *                    chunk routed and appended to its precision segment.
+ *   mq_decode_attn_partial / mq_combine_partials
+ *                    a sequence split by context across devices: per-shard
+ *                    partial results, merged after an all-gather.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -388,6 +391,45 @@ mq_status mq_decode_attn_noalloc(const mq_shape* shape, const int32_t* h_seq_len
                                  const void* layout, const void* packed,
                                  const void* q, int32_t q_dtype, float softmax_scale,
                                  float* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Context split across devices: mq_decode_attn_partial + mq_combine_partials.
+ *
+ * A long sequence can be split by context: device r holds a contiguous range
+ * of whole chunks of every sequence (routed with routing_freeze only on the
+ * device holding chunk 0), builds its own layout and packed cache for that
+ * range, and computes a partial result for every (sequence, query head).
+ * The records of all devices are gathered (an all-gather over NVLink) and
+ * merged with mq_combine_partials.  The merge is the usual split softmax
+ * (the pages are silent on it): with m_r a reference score of shard r and
+ * l_r = sum exp(score - m_r) over its tokens,
+ *     M = max_r m_r,  w_r = l_r exp(m_r - M),  o = sum_r w_r o_r / sum_r w_r.
+ *
+ * Record layout, MQ_PARTIAL_FLOATS(d) floats per (b, h), [B][Hq] order:
+ *     [ o_0 .. o_{d-1} (this shard's normalised output), m, l, 0, 0 ]
+ * m is not necessarily the largest score: the decode moves its reference only
+ * when a score exceeds it by more than 8 ln 2, so the largest score lies in
+ * [m, m + 8 ln 2] and l <= 256 * tokens; m + ln l (the log-sum-exp of the
+ * shard's scores) is what the record fixes.  An empty shard gives m = -inf,
+ * l = 0, o = 0.
+ * ------------------------------------------------------------------------- */
+#define MQ_PARTIAL_FLOATS(d) ((d) + 4)
+
+/* mq_decode_attn over this device's shard, writing records instead of the
+ * output: partial is device fp32 [B, Hq, MQ_PARTIAL_FLOATS(d)].  Other
+ * arguments and errors as mq_decode_attn. */
+mq_status mq_decode_attn_partial(const mq_shape* shape, const int32_t* h_seq_lens,
+                                 const void* layout, const void* packed, const void* q,
+                                 int32_t q_dtype, float softmax_scale, float* partial,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Merges num_parts records per (b, h): partials is device fp32
+ * [num_parts][num_seqs][num_q_heads][MQ_PARTIAL_FLOATS(head_dim)] (the
+ * gathered records, shard order irrelevant), out is device fp32
+ * [num_seqs, num_q_heads, head_dim].  head_dim 64 or 128. */
+mq_status mq_combine_partials(int32_t num_parts, int32_t num_seqs, int32_t num_q_heads,
+                              int32_t head_dim, const float* partials, float* out,
+                              void* stream);
 
 /* ---------------------------------------------------------------------------
  * Cache growth during decoding (mq_grow_*).
