@@ -125,26 +125,32 @@ mq_status report_error(mq_status status, const char* fmt, ...) {
 // ------------------------------------------------------------ item policy
 
 ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens) {
-  // A work item carries about 32 KiB of packed K+V (64 KiB when four or more
-  // query heads share a kv-head, whose per-item partial results are larger),
+  // Work items are balanced by estimated decode time, not by bytes: a token
+  // costs its packed bytes plus a fixed amount of arithmetic (code expansion,
+  // dot products, softmax), about 374 byte-equivalents per query head group
+  // for one query head (fitted to the single-precision decode rates: FP16
+  // 5.2, INT4 2.7, INT2 1.85 TB/s), growing with the query heads that share a
+  // kv-head.  An item carries about 2^17 byte-equivalents (2^19 with four or
+  // more query heads per kv-head, whose per-item partial results are larger)
   // so the partial results stay a few percent of the bytes read.  Small
   // problems are split finer (by powers of two, down to 32 tokens) so that
-  // there are at least ~8 items per SM of a 148-SM part.  Depends only on the
-  // shape and the lengths, so size queries and layout builds agree without a
-  // GPU.
+  // every worker warp of a 148-SM part gets several items.  Depends only on
+  // the shape and the lengths, so size queries and layout builds agree
+  // without a GPU.
   const int d = s.head_dim;
   const int qpg = s.num_q_heads / s.num_kv_heads;
   const int bpt[kNumExperts] = {2 * 2 * d, 2 * (d / 2 + d / 8), 2 * (d / 4 + d / 8)};
-  const int target = 32768 * (qpg >= 4 ? 2 : 1);
+  const int arith = (374 * d / 128) * (2 + 3 * qpg) / 5;  // 0.4 + 0.6 * qpg of one head's
+  const int target = qpg >= 4 ? (1 << 19) : (1 << 17);
   ItemPolicy p;
   for (int e = 0; e < kNumExperts; ++e) {
-    int m = (target / bpt[e]) / 32 * 32;
+    int m = (target / (bpt[e] + arith)) / 32 * 32;
     if (m < 32) m = 32;
     p.item_tokens[e] = m;
   }
   int64_t T = 0;
   for (int b = 0; b < s.num_seqs; ++b) T += h_seq_lens[b];
-  const int64_t want = 148 * 8;
+  const int64_t want = 148 * 2 * 8 * 4;  // worker warps of a 148-SM part x 4
   while (true) {
     const int64_t est = T * s.num_kv_heads / p.item_tokens[1];
     if (est >= want) break;

@@ -11,7 +11,9 @@
 // only — no per-token branching between bitwidths.
 //
 // decode_partial_kernel — every warp is an independent persistent worker
-// that takes work items w = warp id, warp id + total warps, ...  A work item is
+// that takes work items from an atomic counter, one at a time (items differ
+// in cost with their precision, so a static split leaves SMs idle).  A work
+// item is
 // (sequence b, segment s, kv-head g, token range of at most item_tokens[s]
 // tokens).  The warp streams the item's four byte ranges (K codes, V codes, K
 // scales, V scales) through its own 4-stage cp.async ring in shared memory,
@@ -462,15 +464,16 @@ __device__ __forceinline__ int find_item_seq(const unsigned char* layout, int B,
   return lo;
 }
 
-// Each warp is an independent worker: it takes work items w = warp id,
-// warp id + total warps, ... and streams each through its own copy ring.  No
-// block-wide barrier is used.
+// Each warp is an independent worker: it takes the next work item from a
+// counter in the workspace whenever it finishes one, and streams each item
+// through its own copy ring.  No block-wide barrier is used.
 template <int D, int QPG, int QDT>
 __global__ void __launch_bounds__(kDecThreads, 2)
 decode_partial_kernel(const unsigned char* __restrict__ layout,
                       const unsigned char* __restrict__ packed, const void* __restrict__ q,
                       float scale_log2, float* __restrict__ ws_acc, float2* __restrict__ ws_ml,
-                      int64_t capacity_items, unsigned int* status) {
+                      unsigned int* __restrict__ counter, int64_t capacity_items,
+                      unsigned int* status) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
   if (h->magic != MQ_LAYOUT_MAGIC || h->head_dim != D) {
@@ -483,10 +486,15 @@ decode_partial_kernel(const unsigned char* __restrict__ layout,
     if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_WORKSPACE_TOO_SMALL);
     return;
   }
-  const int warp = threadIdx.x / 32;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   unsigned char* ring = smem_raw + (size_t)warp * kRing * stage_bytes<D, QPG>();
-  const int64_t nwarps = (int64_t)gridDim.x * kDecWarps;
-  for (int64_t w = (int64_t)blockIdx.x * kDecWarps + warp; w < total; w += nwarps) {
+  // dynamic assignment: a warp takes the next item when it is done with one,
+  // so items of different cost even out across the SMs
+  for (;;) {
+    unsigned int wi = 0;
+    if (lane == 0) wi = atomicAdd(counter, 1u);
+    const int64_t w = (int64_t)__shfl_sync(0xffffffffu, wi, 0);
+    if (w >= total) break;
     const int64_t bs = w / Hkv;
     const int g = (int)(w - bs * Hkv);
     const int b = find_item_seq(layout, B, bs);
@@ -625,8 +633,9 @@ combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ p
 template <int D, int QPG, int QDT>
 cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layout,
                             const unsigned char* packed, const void* q, float scale_log2,
-                            float* out, float* ws_acc, float2* ws_ml, int num_seqs,
-                            unsigned int* status, cudaStream_t stream, bool partial) {
+                            float* out, float* ws_acc, float2* ws_ml, unsigned int* counter,
+                            int num_seqs, unsigned int* status, cudaStream_t stream,
+                            bool partial) {
   constexpr size_t smem = decode_smem_bytes<D, QPG>();
   auto kern = decode_partial_kernel<D, QPG, QDT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -641,8 +650,10 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
   const int64_t need = (cap + kDecWarps - 1) / kDecWarps;
   if (grid > need) grid = need;
   if (grid > 0) {
+    // worker warps take items from a counter in the workspace, zeroed here
+    if ((err = cudaMemsetAsync(counter, 0, sizeof(unsigned int), stream)) != cudaSuccess) return err;
     kern<<<(unsigned)grid, kDecThreads, smem, stream>>>(layout, packed, q, scale_log2, ws_acc, ws_ml,
-                                                         cap, status);
+                                                         counter, cap, status);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   const int64_t heads = (int64_t)num_seqs * Hq;
@@ -658,13 +669,13 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
 template <int D, int QDT>
 cudaError_t dispatch_qpg(int qpg, int64_t max_items, int Hq, const unsigned char* layout,
                          const unsigned char* packed, const void* q, float scale_log2, float* out,
-                         float* ws_acc, float2* ws_ml, int B, unsigned int* status,
-                         cudaStream_t stream, bool partial) {
+                         float* ws_acc, float2* ws_ml, unsigned int* counter, int B,
+                         unsigned int* status, cudaStream_t stream, bool partial) {
   switch (qpg) {
-    case 1: return launch_decode_t<D, 1, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
-    case 2: return launch_decode_t<D, 2, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
-    case 4: return launch_decode_t<D, 4, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
-    case 8: return launch_decode_t<D, 8, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, B, status, stream, partial);
+    case 1: return launch_decode_t<D, 1, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
+    case 2: return launch_decode_t<D, 2, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
+    case 4: return launch_decode_t<D, 4, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
+    case 8: return launch_decode_t<D, 8, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -674,7 +685,9 @@ cudaError_t dispatch_qpg(int qpg, int64_t max_items, int Hq, const unsigned char
 size_t decode_workspace_bytes(const mq_shape& s, int64_t max_items) {
   const int64_t qpg = s.num_q_heads / s.num_kv_heads;
   const int64_t recs = max_items * s.num_kv_heads * qpg;
-  return (size_t)align128((uint64_t)recs * s.head_dim * 4) + (size_t)align128((uint64_t)recs * 8);
+  // partial (acc) records, (m, l) records, the work counter
+  return (size_t)align128((uint64_t)recs * s.head_dim * 4) + (size_t)align128((uint64_t)recs * 8) +
+         128;
 }
 
 cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layout,
@@ -687,18 +700,21 @@ cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layo
   float* ws_acc = static_cast<float*>(workspace);
   float2* ws_ml = reinterpret_cast<float2*>(static_cast<unsigned char*>(workspace) +
                                             align128((uint64_t)recs * s.head_dim * 4));
+  unsigned int* counter = reinterpret_cast<unsigned int*>(
+      static_cast<unsigned char*>(workspace) + align128((uint64_t)recs * s.head_dim * 4) +
+      align128((uint64_t)recs * 8));
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   const unsigned char* lay = static_cast<const unsigned char*>(layout);
   const unsigned char* pk = static_cast<const unsigned char*>(packed);
   const int64_t cap = max_items * s.num_kv_heads;
   if (s.head_dim == 128) {
     if (q_dtype == MQ_F16)
-      return dispatch_qpg<128, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
-    return dispatch_qpg<128, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
+      return dispatch_qpg<128, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
+    return dispatch_qpg<128, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
   }
   if (q_dtype == MQ_F16)
-    return dispatch_qpg<64, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
-  return dispatch_qpg<64, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, s.num_seqs, status, stream, partial);
+    return dispatch_qpg<64, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
+  return dispatch_qpg<64, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
 }
 
 cudaError_t launch_combine_partials(int P, int B, int Hq, int D, const float* parts, float* out,
