@@ -81,12 +81,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// exact small integer -> float: the integer is OR-ed into the mantissa of
-// 2^23 and 2^23 subtracted again (both steps exact for c < 2^23)
-__device__ __forceinline__ float code_to_float(uint32_t c) {
-  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
-}
-
 __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t bits) {
   __half2 h;
   *reinterpret_cast<uint32_t*>(&h) = bits;
@@ -630,32 +624,492 @@ combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ p
   out[bh * D + i] = den > 0.f ? num / den : 0.f;
 }
 
+// ============================================================================
+// Tensor-core decode for several query heads per kv-head (fp16 queries).
+//
+// With Hq/Hkv = QPG > 1 the CUDA-core kernel above spreads one token over
+// 32/(32/QPG) lanes and repeats the per-token softmax work on each of them.
+// Here a warp takes 16 tokens at a time and lets mma.sync (m16n8k16, fp16
+// operands, fp32 accumulation) form both products:
+//   scores  S[16 tokens x 8 head slots] = Khat . Q^T, one accumulator per group
+//           of 32 dims (the group's scale and min are applied afterwards:
+//           q . khat = s (q . code) + min sum(q));
+//   values  O^T[16 dims x 8 head slots] += Vhat^T . P', P' = p * s_v per group,
+//           P' split into fp16 high and low parts (two MMAs) so that the
+//           products keep fp32-level accuracy; the mins enter as
+//           sum_t p_t min_t per group.
+// Codes become exact fp16 integers (one byte-permute, one mask and one fma
+// per pair).  The dims of a k-step are permuted identically in K and Q so
+// that each lane reads whole bytes: k = 2t, 2t+1, 2t+8, 2t+9 of k-step
+// (group g, half hh) are dims 32g + 8t + 4hh + {0, 1, 2, 3} (t = lane % 4).
+// V codes are expanded into a padded fp16 tile and fed to the MMA with
+// ldmatrix.trans; FP16 segments feed K and V straight from the staged rows.
+// ============================================================================
+constexpr int kMmaWarps = 8;
+constexpr int kMmaThreads = 32 * kMmaWarps;
+constexpr int kMmaTile = 16;            // tokens per tile
+constexpr int kMmaRing = 18 * 1024;     // bytes of one warp's copy ring
+constexpr int kRowPad = 16;             // bytes added to every staged code row
+
+template <int D, int E>
+struct MG {
+  static constexpr int BITS = E == 0 ? 16 : (E == 1 ? 4 : 2);
+  static constexpr int CROW = D * BITS / 8;                 // code bytes of a token row
+  static constexpr int KROW = CROW + kRowPad;               // staged row pitch
+  static constexpr int SROW = E == 0 ? 0 : D / kGroup * 4;  // (scale, min) bytes of a row
+  static constexpr int KOFF = 0;
+  static constexpr int VOFF = kMmaTile * KROW;
+  static constexpr int KSOFF = 2 * kMmaTile * KROW;
+  static constexpr int VSOFF = KSOFF + kMmaTile * SROW;
+  static constexpr int STAGE = (VSOFF + kMmaTile * SROW + 15) / 16 * 16;
+  static constexpr int STAGES = kMmaRing / STAGE < 8 ? kMmaRing / STAGE : 8;
+  // 16-byte copy units of one tile: K codes, V codes, K scales, V scales
+  static constexpr int CU = CROW / 16;                      // units per code row
+  static constexpr int UNITS = 2 * kMmaTile * CU + 2 * SROW;  // a tile's scales: SROW units
+};
+static_assert(MG<128, 0>::STAGES >= 2 && MG<64, 0>::STAGES >= 2, "ring too small");
+
+constexpr int kVbufRow = 128 + 8;       // fp16 elements of one expanded V row (padded)
+constexpr int kVbufBytes = kMmaTile * kVbufRow * 2;
+
+template <int D>
+constexpr size_t mma_smem_bytes() {
+  return (size_t)kMmaWarps * (kMmaRing + kVbufBytes);
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// byte j of w as [b, 0x64, b, 0x64]: two fp16 values 1024 + (low bits of b)
+__device__ __forceinline__ uint32_t spread2(uint32_t w, int j) {
+  return __byte_perm(w, 0x6464u, (uint32_t)j | 0x4000u | ((uint32_t)j << 8) | 0x0050u);
+}
+// INT4: byte j of w -> fp16 pair (low nibble, high nibble), exact
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j) {
+  const __half2 x = bits_h2(spread2(w, j) & 0xFFF0FF0Fu);   // (1024 + lo, 1024 + 16 hi)
+  return h2_bits(__hfma2(x, __floats2half2_rn(1.0f, 0.0625f), __floats2half2_rn(-1024.0f, -64.0f)));
+}
+// INT2: byte j of w -> two fp16 pairs (c0, c1), (c2, c3), exact
+__device__ __forceinline__ void crumb_pairs(uint32_t w, int j, uint32_t& p01, uint32_t& p23) {
+  const uint32_t x = spread2(w, j);
+  p01 = h2_bits(__hfma2(bits_h2(x & 0xFF0CFF03u), __floats2half2_rn(1.0f, 0.25f),
+                        __floats2half2_rn(-1024.0f, -256.0f)));
+  p23 = h2_bits(__hfma2(bits_h2(x & 0xFFC0FF30u), __floats2half2_rn(0.0625f, 0.015625f),
+                        __floats2half2_rn(-64.0f, -16.0f)));
+}
+// fp32 pair -> (high fp16 pair, low fp16 pair) with hi + lo ~ x to ~2^-22
+__device__ __forceinline__ void split_h2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x, y);
+  const float2 hf = __half22float2(h);
+  hi = h2_bits(h);
+  lo = h2_bits(__floats2half2_rn(x - hf.x, y - hf.y));
+}
+
+template <int D, int QPG, int E>
+__device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
+                                         const unsigned char* __restrict__ regv, uint64_t soff,
+                                         int t0, int n, const __half* __restrict__ q, int64_t qbase,
+                                         float scale_log2, unsigned char* ring, __half* vbuf,
+                                         int64_t w, float* __restrict__ ws_acc,
+                                         float2* __restrict__ ws_ml) {
+  using G = MG<D, E>;
+  constexpr int NG = D / 32;  // groups of 32 dims
+  constexpr int NK = D / 16;  // k-steps of the score MMA, m-tiles of O^T
+  constexpr int VROW = D + 8; // fp16 elements of an expanded V row
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+  const int iters = (n + kMmaTile - 1) / kMmaTile;
+
+  // ---- copies of tile `it` into its stage (whole 16-byte units; code rows padded)
+  auto issue = [&](int it) {
+    if (it < iters) {
+      unsigned char* st = ring + (it % G::STAGES) * G::STAGE;
+      const int64_t row0 = t0 + (int64_t)it * kMmaTile;
+      const int nv = min(kMmaTile, n - it * kMmaTile);
+      constexpr int CODE_UNITS = kMmaTile * G::CU;
+      for (int u = lane; u < G::UNITS; u += 32) {
+        if (u < 2 * CODE_UNITS) {
+          const int kv = u >= CODE_UNITS;
+          const int r = u - kv * CODE_UNITS;
+          const int row = r / G::CU, col = (r - row * G::CU) * 16;
+          if (row < nv)
+            cp_async16(st + (kv ? G::VOFF : G::KOFF) + row * G::KROW + col,
+                       (kv ? regv : regk) + (row0 + row) * G::CROW + col);
+        } else if constexpr (E != 0) {
+          const int r = u - 2 * CODE_UNITS;
+          const int kv = r >= G::SROW;           // SROW units of 16 B per tile
+          const int off = (r - kv * G::SROW) * 16;
+          if (off / G::SROW < nv)
+            cp_async16(st + (kv ? G::VSOFF : G::KSOFF) + off,
+                       (kv ? regv : regk) + soff + row0 * G::SROW + off);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll 1
+  for (int it = 0; it < G::STAGES - 1; ++it) issue(it);
+
+  // ---- query operand (B of the score MMA): head slot gid, zero past QPG
+  uint32_t qb[NK][2];
+  float qsum[NG][2];
+  {
+    const bool hv = gid < QPG;
+    const __half* qh = q + qbase + (int64_t)(hv ? gid : 0) * D;
+    float part[NG];
+#pragma unroll
+    for (int g = 0; g < NG; ++g) part[g] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk) {
+      const int d0 = E == 0 ? 16 * kk + 2 * tig : 32 * (kk / 2) + 8 * tig + 4 * (kk % 2);
+      const int d1 = E == 0 ? d0 + 8 : d0 + 2;
+      const uint32_t b0 = hv ? *reinterpret_cast<const uint32_t*>(qh + d0) : 0u;
+      const uint32_t b1 = hv ? *reinterpret_cast<const uint32_t*>(qh + d1) : 0u;
+      qb[kk][0] = b0;
+      qb[kk][1] = b1;
+      const float2 f0 = __half22float2(bits_h2(b0)), f1 = __half22float2(bits_h2(b1));
+      part[kk / 2] += (f0.x + f0.y) + (f1.x + f1.y);
+    }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      part[g] += __shfl_xor_sync(0xffffffffu, part[g], 1);
+      part[g] += __shfl_xor_sync(0xffffffffu, part[g], 2);
+      // sums of heads 2 tig and 2 tig + 1 live in lanes 8 tig and 8 tig + 4
+      qsum[g][0] = __shfl_sync(0xffffffffu, part[g], 8 * tig);
+      qsum[g][1] = __shfl_sync(0xffffffffu, part[g], 8 * tig + 4);
+    }
+  }
+
+  float o[NK][4];
+  float vb[NG][2];
+  float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+#pragma unroll
+  for (int mt = 0; mt < NK; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+#pragma unroll
+  for (int g = 0; g < NG; ++g) vb[g][0] = vb[g][1] = 0.f;
+  const int r0 = gid, r1 = gid + 8;
+
+#pragma unroll 1
+  for (int it = 0; it < iters; ++it) {
+    issue(it + G::STAGES - 1);
+    cp_async_wait<G::STAGES - 1>();
+    __syncwarp();
+    unsigned char* st = ring + (it % G::STAGES) * G::STAGE;
+    const int nv = min(kMmaTile, n - it * kMmaTile);
+    const bool v0 = r0 < nv, v1 = r1 < nv;
+
+    // ---- scores: C rows = tokens (r0, r1), columns = head slots (2 tig, 2 tig + 1)
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (E == 0) {
+      const uint32_t kbase = smem_addr(st + G::KOFF);
+      const int j = lane >> 3;
+      const uint32_t arow = kbase + ((lane & 7) + (j & 1) * 8) * G::KROW + (j >> 1) * 16;
+#pragma unroll
+      for (int kk = 0; kk < NK; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(a, arow + kk * 32);
+        mma16816(s4, a[0], a[1], a[2], a[3], qb[kk][0], qb[kk][1]);
+      }
+    } else {
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (E == 1) {
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(st + G::KOFF + r0 * G::KROW + 4 * (4 * g + tig));
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(st + G::KOFF + r1 * G::KROW + 4 * (4 * g + tig));
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            mma16816(acc, nib_pair(w0, 2 * hh), nib_pair(w1, 2 * hh), nib_pair(w0, 2 * hh + 1),
+                     nib_pair(w1, 2 * hh + 1), qb[2 * g + hh][0], qb[2 * g + hh][1]);
+        } else {
+          const uint32_t h0 = *reinterpret_cast<const unsigned short*>(st + G::KOFF + r0 * G::KROW + 8 * g + 2 * tig);
+          const uint32_t h1 = *reinterpret_cast<const unsigned short*>(st + G::KOFF + r1 * G::KROW + 8 * g + 2 * tig);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t a0, a2, a1, a3;
+            crumb_pairs(h0, hh, a0, a2);
+            crumb_pairs(h1, hh, a1, a3);
+            mma16816(acc, a0, a1, a2, a3, qb[2 * g + hh][0], qb[2 * g + hh][1]);
+          }
+        }
+        const float2 sm0 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r0 * G::SROW + 4 * g));
+        const float2 sm1 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r1 * G::SROW + 4 * g));
+        s4[0] = fmaf(sm0.x, acc[0], fmaf(sm0.y, qsum[g][0], s4[0]));
+        s4[1] = fmaf(sm0.x, acc[1], fmaf(sm0.y, qsum[g][1], s4[1]));
+        s4[2] = fmaf(sm1.x, acc[2], fmaf(sm1.y, qsum[g][0], s4[2]));
+        s4[3] = fmaf(sm1.x, acc[3], fmaf(sm1.y, qsum[g][1], s4[3]));
+      }
+    }
+
+    // ---- online softmax per head slot (log2 domain, lazily moved reference;
+    // rows past the item's end hold stale bytes and are masked, never used)
+    float sc[4];
+    sc[0] = v0 ? s4[0] * scale_log2 : -INFINITY;
+    sc[1] = v0 ? s4[1] * scale_log2 : -INFINITY;
+    sc[2] = v1 ? s4[2] * scale_log2 : -INFINITY;
+    sc[3] = v1 ? s4[3] * scale_log2 : -INFINITY;
+    float tm[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      tm[0] = fmaxf(tm[0], __shfl_xor_sync(0xffffffffu, tm[0], off));
+      tm[1] = fmaxf(tm[1], __shfl_xor_sync(0xffffffffu, tm[1], off));
+    }
+#pragma unroll
+    for (int hj = 0; hj < 2; ++hj) {
+      if (tm[hj] > mrun[hj] + kRescale) {
+        const float a = exp2f(mrun[hj] - tm[hj]);
+        lsum[hj] *= a;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) vb[g][hj] *= a;
+#pragma unroll
+        for (int mt = 0; mt < NK; ++mt) {
+          o[mt][hj] *= a;
+          o[mt][2 + hj] *= a;
+        }
+        mrun[hj] = tm[hj];
+      }
+    }
+    float p[4];
+    p[0] = v0 ? exp2f(sc[0] - mrun[0]) : 0.f;
+    p[1] = v0 ? exp2f(sc[1] - mrun[1]) : 0.f;
+    p[2] = v1 ? exp2f(sc[2] - mrun[0]) : 0.f;
+    p[3] = v1 ? exp2f(sc[3] - mrun[1]) : 0.f;
+    lsum[0] += p[0] + p[2];
+    lsum[1] += p[1] + p[3];
+
+    // ---- values: O^T[dims x head slots] += Vhat^T . P'
+    if constexpr (E != 0) {
+      // expand this tile's V codes into vbuf (natural dim order), two lanes a row
+      {
+        const int row = lane >> 1, half = lane & 1;
+        constexpr int HB = G::CROW / 2;  // code bytes of half a row
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(st + G::VOFF + row * G::KROW + half * HB);
+        __half* dst = vbuf + row * VROW + half * (HB * 8 / G::BITS);
+#pragma unroll
+        for (int k = 0; k < HB / 4; ++k) {
+          const uint32_t wv = src[k];
+          if constexpr (E == 1) {
+            *reinterpret_cast<uint4*>(dst + 8 * k) =
+                make_uint4(nib_pair(wv, 0), nib_pair(wv, 1), nib_pair(wv, 2), nib_pair(wv, 3));
+          } else {
+            uint32_t c[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) crumb_pairs(wv, j, c[2 * j], c[2 * j + 1]);
+            *reinterpret_cast<uint4*>(dst + 16 * k) = make_uint4(c[0], c[1], c[2], c[3]);
+            *reinterpret_cast<uint4*>(dst + 16 * k + 8) = make_uint4(c[4], c[5], c[6], c[7]);
+          }
+        }
+      }
+      __syncwarp();
+      const uint32_t vbase = smem_addr(vbuf);
+      const int j = lane >> 3;
+      const uint32_t arow = vbase + ((lane & 7) + (j >> 1) * 8) * (VROW * 2) + (j & 1) * 16;
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const float2 sm0 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r0 * G::SROW + 4 * g));
+        const float2 sm1 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r1 * G::SROW + 4 * g));
+        // p * scale per token, divided by 2^E with 2^E <= the tile's largest
+        // scale of this group so that it fits fp16 (p <= 2^8, scale <= 65504);
+        // the MMA result is multiplied back by 2^E (both exact).  Rows past
+        // the item's end contribute exactly 0, never 0 * stale bytes.
+        float smax = fmaxf(v0 ? sm0.x : 0.f, v1 ? sm1.x : 0.f);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+        const uint32_t eb = __float_as_uint(smax) & 0x7F800000u;       // 2^E (E = floor(log2 smax))
+        const float up = eb ? __uint_as_float(eb) : 1.f;
+        const float down = eb ? __uint_as_float(0x7F000000u - eb) : 1.f; // 2^-E
+        const float s0 = sm0.x * down, s1 = sm1.x * down;
+        const float x0 = v0 ? p[0] * s0 : 0.f, x1 = v0 ? p[1] * s0 : 0.f;
+        const float x2 = v1 ? p[2] * s1 : 0.f, x3 = v1 ? p[3] * s1 : 0.f;
+        vb[g][0] += (v0 ? p[0] * sm0.y : 0.f) + (v1 ? p[2] * sm1.y : 0.f);
+        vb[g][1] += (v0 ? p[1] * sm0.y : 0.f) + (v1 ? p[3] * sm1.y : 0.f);
+        uint32_t hi0, lo0, hi1, lo1;
+        split_h2(x0, x1, hi0, lo0);
+        split_h2(x2, x3, hi1, lo1);
+        const uint32_t bh0 = movm_t(hi0), bh1 = movm_t(hi1), bl0 = movm_t(lo0), bl1 = movm_t(lo1);
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm) {
+          const int mt = 2 * g + mm;
+          uint32_t a[4];
+          ldsm_x4_t(a, arow + mt * 32);
+          float t[4] = {0.f, 0.f, 0.f, 0.f};
+          mma16816(t, a[0], a[1], a[2], a[3], bh0, bh1);
+          mma16816(t, a[0], a[1], a[2], a[3], bl0, bl1);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[mt][i] = fmaf(up, t[i], o[mt][i]);
+        }
+      }
+    } else {
+      // FP16 rows straight from the stage; rows past the item's end are zeroed
+      // first (stale bytes there need not be numbers, and 0 * NaN is NaN)
+      if (nv < kMmaTile) {
+        constexpr int RU = D * 2 / 16;  // 16-byte units of a row
+        for (int u = lane; u < (kMmaTile - nv) * RU; u += 32) {
+          const int row = nv + u / RU;
+          *reinterpret_cast<uint4*>(st + G::VOFF + row * G::KROW + (u % RU) * 16) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      uint32_t hi0, lo0, hi1, lo1;
+      split_h2(p[0], p[1], hi0, lo0);
+      split_h2(p[2], p[3], hi1, lo1);
+      const uint32_t bh0 = movm_t(hi0), bh1 = movm_t(hi1), bl0 = movm_t(lo0), bl1 = movm_t(lo1);
+      const uint32_t vbase = smem_addr(st + G::VOFF);
+      const int j = lane >> 3;
+      const uint32_t arow = vbase + ((lane & 7) + (j >> 1) * 8) * G::KROW + (j & 1) * 16;
+#pragma unroll
+      for (int mt = 0; mt < NK; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_t(a, arow + mt * 32);
+        mma16816(o[mt], a[0], a[1], a[2], a[3], bh0, bh1);
+        mma16816(o[mt], a[0], a[1], a[2], a[3], bl0, bl1);
+      }
+    }
+    __syncwarp();  // the stage and vbuf are read before they are refilled
+  }
+  cp_async_wait<0>();
+
+  // ---- partial results of the item: sum over the token lanes, then per head slot
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], off);
+    lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], off);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      vb[g][0] += __shfl_xor_sync(0xffffffffu, vb[g][0], off);
+      vb[g][1] += __shfl_xor_sync(0xffffffffu, vb[g][1], off);
+    }
+  }
+#pragma unroll
+  for (int hj = 0; hj < 2; ++hj) {
+    const int h = 2 * tig + hj;
+    if (h < QPG) {
+      float* dst = ws_acc + ((size_t)w * QPG + h) * D;
+#pragma unroll
+      for (int mt = 0; mt < NK; ++mt) {
+        const int d0 = 16 * mt + gid, d1 = d0 + 8;
+        dst[d0] = o[mt][hj] + vb[d0 / 32][hj];
+        dst[d1] = o[mt][2 + hj] + vb[d1 / 32][hj];
+      }
+      if (gid == 0) ws_ml[(size_t)w * QPG + h] = make_float2(mrun[hj], lsum[hj]);
+    }
+  }
+  __syncwarp();
+}
+
+template <int D, int QPG>
+__global__ void __launch_bounds__(kMmaThreads, 1)
+decode_mma_kernel(const unsigned char* __restrict__ layout, const unsigned char* __restrict__ packed,
+                  const __half* __restrict__ q, float scale_log2, float* __restrict__ ws_acc,
+                  float2* __restrict__ ws_ml, unsigned int* __restrict__ counter,
+                  int64_t capacity_items, unsigned int* status) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
+  if (h->magic != MQ_LAYOUT_MAGIC || h->head_dim != D) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_BAD_LAYOUT);
+    return;
+  }
+  const int B = h->num_seqs, Hkv = h->num_kv_heads;
+  const int64_t total = (int64_t)h->total_items * Hkv;
+  if (total > capacity_items) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_WORKSPACE_TOO_SMALL);
+    return;
+  }
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  unsigned char* ring = smem_raw + (size_t)warp * (kMmaRing + kVbufBytes);
+  __half* vbuf = reinterpret_cast<__half*>(ring + kMmaRing);
+  for (;;) {
+    unsigned int wi = 0;
+    if (lane == 0) wi = atomicAdd(counter, 1u);
+    const int64_t w = (int64_t)__shfl_sync(0xffffffffu, wi, 0);
+    if (w >= total) break;
+    const int64_t bs = w / Hkv;
+    const int g = (int)(w - bs * Hkv);
+    const int b = find_item_seq(layout, B, bs);
+    const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
+    const int s = bs < r->item_begin[1] ? 0 : (bs < r->item_begin[2] ? 1 : 2);
+    const int j = (int)(bs - r->item_begin[s]);
+    const int t0 = j * h->item_tokens[s];
+    const int n = min(h->item_tokens[s], r->seg_tokens[s] - t0);
+    if (n <= 0) {
+      if (lane == 0) set_status(status, MQ_DEV_INDEX_RANGE);
+      continue;
+    }
+    const unsigned char* regk = packed + r->seg_base[s] + (uint64_t)g * r->region_bytes[s];
+    const unsigned char* regv = regk + (uint64_t)Hkv * r->region_bytes[s];
+    const int64_t qbase = ((int64_t)b * Hkv + g) * QPG * D;
+    if (s == 0)
+      mma_item<D, QPG, 0>(regk, regv, 0, t0, n, q, qbase, scale_log2, ring, vbuf, w, ws_acc, ws_ml);
+    else if (s == 1)
+      mma_item<D, QPG, 1>(regk, regv, r->scale_offset[1], t0, n, q, qbase, scale_log2, ring, vbuf,
+                          w, ws_acc, ws_ml);
+    else
+      mma_item<D, QPG, 2>(regk, regv, r->scale_offset[2], t0, n, q, qbase, scale_log2, ring, vbuf,
+                          w, ws_acc, ws_ml);
+  }
+}
+
 template <int D, int QPG, int QDT>
 cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layout,
                             const unsigned char* packed, const void* q, float scale_log2,
                             float* out, float* ws_acc, float2* ws_ml, unsigned int* counter,
                             int num_seqs, unsigned int* status, cudaStream_t stream,
                             bool partial) {
-  constexpr size_t smem = decode_smem_bytes<D, QPG>();
-  auto kern = decode_partial_kernel<D, QPG, QDT>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
+  // several query heads per kv-head with fp16 queries: the tensor-core kernel
+  constexpr bool kMma = QDT == MQ_F16 && QPG >= 2;
+  constexpr size_t smem = kMma ? mma_smem_bytes<D>() : decode_smem_bytes<D, QPG>();
+  constexpr int threads = kMma ? kMmaThreads : kDecThreads;
+  constexpr int warps = kMma ? kMmaWarps : kDecWarps;
+  cudaError_t err;
   int dev = 0, sms = 0, per_sm = 0;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
-  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem)) != cudaSuccess)
-    return err;
   const int64_t cap = max_items;  // work items x kv-heads the workspace holds
-  int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
-  const int64_t need = (cap + kDecWarps - 1) / kDecWarps;
-  if (grid > need) grid = need;
-  if (grid > 0) {
-    // worker warps take items from a counter in the workspace, zeroed here
-    if ((err = cudaMemsetAsync(counter, 0, sizeof(unsigned int), stream)) != cudaSuccess) return err;
-    kern<<<(unsigned)grid, kDecThreads, smem, stream>>>(layout, packed, q, scale_log2, ws_acc, ws_ml,
-                                                         counter, cap, status);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  }
+  auto run = [&](auto kern, auto qptr) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem)) != cudaSuccess)
+      return e;
+    int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    const int64_t need = (cap + warps - 1) / warps;
+    if (grid > need) grid = need;
+    if (grid > 0) {
+      // worker warps take items from a counter in the workspace, zeroed here
+      if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned int), stream)) != cudaSuccess) return e;
+      kern<<<(unsigned)grid, threads, smem, stream>>>(layout, packed, qptr, scale_log2, ws_acc, ws_ml,
+                                                      counter, cap, status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  };
+  if constexpr (kMma)
+    err = run(decode_mma_kernel<D, QPG>, static_cast<const __half*>(q));
+  else
+    err = run(decode_partial_kernel<D, QPG, QDT>, q);
+  if (err != cudaSuccess) return err;
   const int64_t heads = (int64_t)num_seqs * Hq;
   if (partial)
     decode_combine_kernel<D, QPG, true><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc,

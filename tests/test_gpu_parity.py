@@ -27,6 +27,9 @@ CASES = {
     "short_chunks": Case(np.array([2048, 33], np.int32), 16, 16, 128, 32),
     "gqa8_d64_L256": Case(np.array([5000, 257], np.int32), 8, 1, 64, 256),
     "gqa2_f32": Case(np.array([700, 64, 1], np.int32), 4, 2, 128, 64, "f32"),
+    "gqa2_f16": Case(np.array([700, 64, 1, 0], np.int32), 4, 2, 128, 64, "f16"),
+    "gqa8_d128": Case(np.array([2000, 33], np.int32), 16, 2, 128, 128, "f16"),
+    "gqa4_d64": Case(np.array([1500, 17, 96], np.int32), 8, 2, 64, 32, "f16"),
 }
 
 MAPS = {"mixed": (0.2, 0.5, 0.3), "fp16": (1, 0, 0), "int4": (0, 1, 0), "int2": (0, 0, 1)}
@@ -40,7 +43,7 @@ def _map(case, mix, seed=0):
 @pytest.mark.parametrize("mapname", list(MAPS))
 def test_layout_pack_decode_parity(name, mapname):
     case = CASES[name]
-    if mapname != "mixed" and name not in ("ragged_gqa4", "tiny_like_f32"):
+    if mapname != "mixed" and name not in ("ragged_gqa4", "tiny_like_f32", "gqa8_d128", "gqa4_d64"):
         pytest.skip("single-precision maps run on two cases")
     cmap = _map(case, MAPS[mapname], seed=zlib.crc32(name.encode()) & 0xFFFF)
     K, V, q = random_kv(case, seed=len(name))
@@ -267,3 +270,24 @@ def test_pack_adversarial_values_bit_exact(dtype):
         if not np.array_equal(got, ref):
             bad = np.nonzero(got != ref)[0]
             raise AssertionError(f"{mapname}: {len(bad)} packed bytes differ, first at {bad[:8]}")
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (4, 4)])
+def test_decode_with_very_large_groups(hq, hkv):
+    # groups whose range reaches ~6e4 (scale ~4e4 at INT2): products of softmax
+    # weights and scales far beyond fp16 range must not overflow anywhere
+    case = Case(np.array([900, 130], np.int32), hq, hkv, 128, 64, "f16")
+    K, V, q = random_kv(case, seed=77)
+    g = torch.Generator().manual_seed(78)
+    big = torch.rand(case.T, case.Hkv, 1, generator=g) < 0.3
+    V = torch.where(big, (V.float() * 20000).clamp(-65000, 65000), V.float()).half()
+    K = (K.float() * 0.05).half()
+    cmap = _map(case, MAPS["mixed"], seed=5)
+    layout = gpu_layout(case, cmap)
+    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+    ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, K.numpy(), V.numpy())
+    assert np.array_equal(packed[:pb].cpu().numpy(), ref)
+    out = gpu_decode(case, layout, packed, q.to(dev()))
+    want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
+    scale = np.abs(want).max()
+    check_attention(out / scale, want / scale, "large groups (relative to the output range)")
