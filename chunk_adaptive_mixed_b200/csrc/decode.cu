@@ -636,8 +636,9 @@ combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ p
 //           q . khat = s (q . code) + min sum(q));
 //   values  O^T[16 dims x 8 head slots] += Vhat^T . P', P' = p * s_v per group,
 //           P' split into fp16 high and low parts (two MMAs) so that the
-//           products keep fp32-level accuracy; the mins enter as
-//           sum_t p_t min_t per group.
+//           products keep fp32-level accuracy, O held in units of a power
+//           of two raised with the largest scale seen so P' fits fp16; the
+//           mins enter as sum_t p_t min_t per group.
 // Codes become exact fp16 integers (one byte-permute, one mask and one fma
 // per pair).  The dims of a k-step are permuted identically in K and Q so
 // that each lane reads whole bytes: k = 2t, 2t+1, 2t+8, 2t+9 of k-step
@@ -645,10 +646,10 @@ combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ p
 // V codes are expanded into a padded fp16 tile and fed to the MMA with
 // ldmatrix.trans; FP16 segments feed K and V straight from the staged rows.
 // ============================================================================
-constexpr int kMmaWarps = 8;
+constexpr int kMmaWarps = 1;            // one worker warp per CTA: ~10 resident per SM
 constexpr int kMmaThreads = 32 * kMmaWarps;
 constexpr int kMmaTile = 16;            // tokens per tile
-constexpr int kMmaRing = 18 * 1024;     // bytes of one warp's copy ring
+constexpr int kMmaRing = 17408;         // bytes of one warp's copy ring (2 FP16 tiles at d=128)
 constexpr int kRowPad = 16;             // bytes added to every staged code row
 
 template <int D, int E>
@@ -743,25 +744,32 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
   const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
   const int iters = (n + kMmaTile - 1) / kMmaTile;
 
-  // ---- copies of tile `it` into its stage (whole 16-byte units; code rows padded)
+  // ---- copies of tile `it` into its stage (whole 16-byte units; code rows
+  // padded): each lane keeps one column of the rows and steps over rows
+  constexpr int RPI = 32 / G::CU;                  // rows per pass of the warp
+  constexpr int PASSES = RPI >= kMmaTile ? 1 : kMmaTile / RPI;
+  const int lrow = lane / G::CU, lcol = (lane % G::CU) * 16;
   auto issue = [&](int it) {
     if (it < iters) {
       unsigned char* st = ring + (it % G::STAGES) * G::STAGE;
       const int64_t row0 = t0 + (int64_t)it * kMmaTile;
       const int nv = min(kMmaTile, n - it * kMmaTile);
-      constexpr int CODE_UNITS = kMmaTile * G::CU;
-      for (int u = lane; u < G::UNITS; u += 32) {
-        if (u < 2 * CODE_UNITS) {
-          const int kv = u >= CODE_UNITS;
-          const int r = u - kv * CODE_UNITS;
-          const int row = r / G::CU, col = (r - row * G::CU) * 16;
-          if (row < nv)
-            cp_async16(st + (kv ? G::VOFF : G::KOFF) + row * G::KROW + col,
-                       (kv ? regv : regk) + (row0 + row) * G::CROW + col);
-        } else if constexpr (E != 0) {
-          const int r = u - 2 * CODE_UNITS;
-          const int kv = r >= G::SROW;           // SROW units of 16 B per tile
-          const int off = (r - kv * G::SROW) * 16;
+      const unsigned char* sk = regk + (row0 + lrow) * G::CROW + lcol;
+      const unsigned char* sv = regv + (row0 + lrow) * G::CROW + lcol;
+      unsigned char* dk = st + G::KOFF + lrow * G::KROW + lcol;
+      unsigned char* dv = st + G::VOFF + lrow * G::KROW + lcol;
+#pragma unroll
+      for (int i = 0; i < PASSES; ++i) {
+        if (lrow + i * RPI < nv) {
+          cp_async16(dk + i * RPI * G::KROW, sk + i * RPI * G::CROW);
+          cp_async16(dv + i * RPI * G::KROW, sv + i * RPI * G::CROW);
+        }
+      }
+      if constexpr (E != 0) {
+        // a tile's scales are SROW 16-byte units per array (K, then V)
+        if (lane < 2 * G::SROW) {
+          const int kv = lane >= G::SROW;
+          const int off = (lane - kv * G::SROW) * 16;
           if (off / G::SROW < nv)
             cp_async16(st + (kv ? G::VSOFF : G::KSOFF) + off,
                        (kv ? regv : regk) + soff + row0 * G::SROW + off);
@@ -806,6 +814,9 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
   float o[NK][4];
   float vb[NG][2];
   float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+  // INT items hold O in units of 2^A (abits = bits of 2^A; 0 until the first
+  // nonzero scale sets A to its binade); FP16 items in plain units
+  uint32_t abits = 0u;
 #pragma unroll
   for (int mt = 0; mt < NK; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 #pragma unroll
@@ -927,20 +938,36 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
       const uint32_t vbase = smem_addr(vbuf);
       const int j = lane >> 3;
       const uint32_t arow = vbase + ((lane & 7) + (j >> 1) * 8) * (VROW * 2) + (j & 1) * 16;
+      // O is kept in units of 2^A, A raised (like the softmax reference) when
+      // a tile brings a scale of a higher binade, so that p * scale * 2^-A
+      // stays within fp16 (p <= 2^8, scale <= 65504); both rescalings are
+      // exact powers of two
+      float2 vsm[NG][2];
+      float smax = 0.f;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
-        const float2 sm0 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r0 * G::SROW + 4 * g));
-        const float2 sm1 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r1 * G::SROW + 4 * g));
-        // p * scale per token, divided by 2^E with 2^E <= the tile's largest
-        // scale of this group so that it fits fp16 (p <= 2^8, scale <= 65504);
-        // the MMA result is multiplied back by 2^E (both exact).  Rows past
-        // the item's end contribute exactly 0, never 0 * stale bytes.
-        float smax = fmaxf(v0 ? sm0.x : 0.f, v1 ? sm1.x : 0.f);
+        vsm[g][0] = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r0 * G::SROW + 4 * g));
+        vsm[g][1] = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r1 * G::SROW + 4 * g));
+        smax = fmaxf(smax, fmaxf(v0 ? vsm[g][0].x : 0.f, v1 ? vsm[g][1].x : 0.f));
+      }
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
-        const uint32_t eb = __float_as_uint(smax) & 0x7F800000u;       // 2^E (E = floor(log2 smax))
-        const float up = eb ? __uint_as_float(eb) : 1.f;
-        const float down = eb ? __uint_as_float(0x7F000000u - eb) : 1.f; // 2^-E
+      for (int off = 4; off < 32; off <<= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+      const uint32_t eb = __float_as_uint(smax) & 0x7F800000u;
+      if (eb > abits) {  // uniform over the warp
+        if (abits != 0u) {
+          const float f = __uint_as_float(0x3F800000u + abits - eb);  // 2^(A_old - A_new)
+#pragma unroll
+          for (int mt = 0; mt < NK; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[mt][i] *= f;
+        }
+        abits = eb;
+      }
+      const float down = __uint_as_float(0x7F000000u - abits);  // 2^-A
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        const float2 sm0 = vsm[g][0], sm1 = vsm[g][1];
+        // rows past the item's end contribute exactly 0, never 0 * stale bytes
         const float s0 = sm0.x * down, s1 = sm1.x * down;
         const float x0 = v0 ? p[0] * s0 : 0.f, x1 = v0 ? p[1] * s0 : 0.f;
         const float x2 = v1 ? p[2] * s1 : 0.f, x3 = v1 ? p[3] * s1 : 0.f;
@@ -955,11 +982,8 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
           const int mt = 2 * g + mm;
           uint32_t a[4];
           ldsm_x4_t(a, arow + mt * 32);
-          float t[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(t, a[0], a[1], a[2], a[3], bh0, bh1);
-          mma16816(t, a[0], a[1], a[2], a[3], bl0, bl1);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[mt][i] = fmaf(up, t[i], o[mt][i]);
+          mma16816(o[mt], a[0], a[1], a[2], a[3], bh0, bh1);
+          mma16816(o[mt], a[0], a[1], a[2], a[3], bl0, bl1);
         }
       }
     } else {
@@ -1004,6 +1028,7 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
     }
   }
 #pragma unroll
+  const float up = (E == 0 || abits == 0u) ? 1.f : __uint_as_float(abits);  // 2^A
   for (int hj = 0; hj < 2; ++hj) {
     const int h = 2 * tig + hj;
     if (h < QPG) {
@@ -1011,8 +1036,8 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
 #pragma unroll
       for (int mt = 0; mt < NK; ++mt) {
         const int d0 = 16 * mt + gid, d1 = d0 + 8;
-        dst[d0] = o[mt][hj] + vb[d0 / 32][hj];
-        dst[d1] = o[mt][2 + hj] + vb[d1 / 32][hj];
+        dst[d0] = fmaf(o[mt][hj], up, vb[d0 / 32][hj]);
+        dst[d1] = fmaf(o[mt][2 + hj], up, vb[d1 / 32][hj]);
       }
       if (gid == 0) ws_ml[(size_t)w * QPG + h] = make_float2(mrun[hj], lsum[hj]);
     }
@@ -1021,7 +1046,7 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
 }
 
 template <int D, int QPG>
-__global__ void __launch_bounds__(kMmaThreads, 1)
+__global__ void __launch_bounds__(kMmaThreads, 10)
 decode_mma_kernel(const unsigned char* __restrict__ layout, const unsigned char* __restrict__ packed,
                   const __half* __restrict__ q, float scale_log2, float* __restrict__ ws_acc,
                   float2* __restrict__ ws_ml, unsigned int* __restrict__ counter,

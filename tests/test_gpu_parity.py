@@ -291,3 +291,18 @@ def test_decode_with_very_large_groups(hq, hkv):
     want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
     scale = np.abs(want).max()
     check_attention(out / scale, want / scale, "large groups (relative to the output range)")
+
+
+def test_decode_with_tiny_values():
+    # every group tiny (scales ~1e-6): the tensor-core path keeps its relative accuracy
+    case = Case(np.array([700, 90], np.int32), 8, 2, 128, 64, "f16")
+    K, V, q = random_kv(case, seed=91)
+    V = (V.float() * 2e-5).half()
+    cmap = _map(case, MAPS["mixed"], seed=6)
+    layout = gpu_layout(case, cmap)
+    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+    ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, K.numpy(), V.numpy())
+    out = gpu_decode(case, layout, packed, q.to(dev()))
+    want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
+    scale = np.abs(want).max()
+    check_attention(out / scale, want / scale, "tiny values (relative to the output range)")
