@@ -107,16 +107,14 @@ def pack_traffic(w, S, seed):
 
 
 def peaks_all():
-    """{hbm GB/s, tf32 TFLOP/s}: the measured copy bandwidth, and the measured
-    bf16 GEMM burst rate times the nominal dense tf32/bf16 ratio (1.1 / 2.25)."""
+    """{hbm GB/s, bf16 TFLOP/s}: the measured copy bandwidth and the measured
+    bf16 GEMM burst rate (the router's MMAs are bf16)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return {"hbm": float(d["hbm_gbs"]), "tf32": float(d["bf16_tflops"]) * 1.1 / 2.25,
-                "source": "measured (tf32 = measured bf16 x nominal 1.1/2.25)"}
-    return {"hbm": 6650.0, "tf32": 1590.0 * 1.1 / 2.25,
-            "source": "fallback (tf32 = fallback bf16 x nominal 1.1/2.25)"}
+        return {"hbm": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "source": "fallback"}
 
 
 def route_summary(S, route_ms, peaks):
@@ -124,13 +122,15 @@ def route_summary(S, route_ms, peaks):
     amount, unit, bound = S.route_work()
     maps = len(S.routers)
     rate = amount * maps / (route_ms / 1e3) / (1e9 if unit == "GB/s" else 1e12)
-    peak = peaks["hbm"] if bound == "hbm" else peaks["tf32"]
+    peak = peaks["hbm"] if bound == "hbm" else peaks["bf16"]
     out = {"router": S.router, "maps_per_step": maps, "avg_ms_per_step": route_ms,
            "achieved": rate, "unit": unit, "bound": bound, "peak": peak, "frac": rate / peak,
            "peak_source": peaks["source"],
            "algorithmic_per_map": amount, "includes": "map kernels only (layout excluded)"}
     if bound == "tensor":
-        out["tensor_passes"] = 3   # tf32 hi*hi + hi*lo + lo*hi: 3x the algorithmic MMAs
+        # bf16 hi*hi + hi*lo + lo*hi: the tensor cores do 3x the algorithmic work
+        out["tensor_passes"] = 3
+        out["tensor_frac"] = 3 * rate / peak
     return out
 
 

@@ -4,11 +4,11 @@
 // chunk C is scored against the experts {FP16, INT4, INT2} by a small MLP,
 // read here as z_t = (SiLU(C_t W1) ⊙ (C_t W2)) W3 + b3.  The two projections
 // C·W1 and C·W2 are one dense contraction [T, D] x [D, 2H]: it runs on
-// tcgen05.mma (kind::tf32) with fp32-equivalent accuracy by splitting both
-// operands into a tf32 high part and an fp32 remainder (x = hi + lo) and
-// accumulating hi·hi + hi·lo + lo·hi (the dropped lo·lo term and the tf32
-// truncation of lo leave a relative error near 2^-21 per product, below the
-// rounding of a plain fp32 dot product of length D).
+// tcgen05.mma (kind::f16 with bf16 operands) by splitting both operands into
+// a bf16 high part and the bf16 of the remainder (x ~ hi + lo) and
+// accumulating hi·hi + hi·lo + lo·hi in fp32 (the dropped lo·lo term and the
+// rounding of lo leave about 2^-16 relative per product; the scores stay
+// within the tolerance the routing decisions allow, see include/mqkv.h).
 //
 // router_tc_kernel: one CTA owns 128 tokens and one block of HB hidden units
 // of both branches (an N = 2*HB accumulator in tensor memory).
@@ -21,13 +21,15 @@
 // Two shared-memory stages; full/empty mbarriers; tcgen05.commit frees a
 // stage when its MMAs complete.  Every wait is bounded: on timeout the kernel
 // records MQ_DEV_WAIT_TIMEOUT, stops, frees its tensor memory and returns.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace mqkv {
 namespace {
 
 constexpr int kTcBM = 128;     // tokens per CTA (MMA M)
-constexpr int kTcBK = 32;      // fp32 elements per k-tile row = one 128-byte swizzle row
+constexpr int kTcKE = 64;      // bf16 k elements per k-tile (one 128-byte swizzle row)
 constexpr int kTcStages = 2;
 constexpr int kTcThreads = 192;
 constexpr uint32_t kTcWaitLimit = 1u << 24;
@@ -94,11 +96,11 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
-__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
@@ -125,12 +127,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// tf32 high part (round to nearest, ties away) and the exact fp32 remainder.
-__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
-  uint32_t h;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
-  hi = __uint_as_float(h);
-  lo = x - hi;
+// bf16 high parts of (a, b) and the bf16 of their remainders, packed in pairs.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // Byte offset of 16-byte chunk c (0..7) of row r inside a K-major tile with
@@ -146,10 +149,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor: fp32 accumulate, tf32 A and B, both K-major.
+// Instruction descriptor: fp32 accumulate, bf16 A and B, both K-major.
 template <int M, int N>
-constexpr uint32_t idesc_tf32() {
-  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 template <int BN>
@@ -174,16 +177,18 @@ __global__ void prepack_weights_kernel(const float* __restrict__ W1, const float
     const int n = q / 8, c = q % 8;
     const float* W = n < HB ? W1 : W2;
     const int col = hb * HB + (n < HB ? n : n - HB);
-    float hi[4], lo[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int k = kt * kTcBK + 4 * c + i;
-      const float x = k < D ? W[(size_t)k * H + col] : 0.0f;
-      split_tf32(x, hi[i], lo[i]);
-    }
     const uint32_t off = swz_off(n, c);
-    *reinterpret_cast<float4*>(tile_hi + off) = make_float4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<float4*>(tile_lo + off) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = kt * kTcKE + 8 * c + i;
+      x[i] = k < D ? W[(size_t)k * H + col] : 0.0f;
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split_bf16x2(x[2 * i], x[2 * i + 1], hi[i], lo[i]);
+    *reinterpret_cast<uint4*>(tile_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(tile_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -237,18 +242,23 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   };
 
   if (warp < 4) {
-    // ---- producers: C tile (128 rows x 32 fp32) -> split -> swizzled stores
+    // ---- producers: C tile (128 rows x kTcKE fp32) -> split -> swizzled stores
     const int t = threadIdx.x;  // 0..127
-    float4 buf[8];
+    constexpr int NV = kTcKE / 32;  // float4 loads per 16-byte chunk of a part
+    float4 buf[8 * NV];
     auto load = [&](int kt) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int f = t + 128 * i;
         const int row = f >> 3, c = f & 7;
         const int64_t tok = m0 + row;
-        const int k = kt * kTcBK + 4 * c;
-        buf[i] = (tok < T && k < D) ? __ldg(reinterpret_cast<const float4*>(C + tok * D + k))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          const int k = kt * kTcKE + (kTcKE / 8) * c + 4 * v;
+          buf[NV * i + v] = (tok < T && k < D)
+                                ? __ldg(reinterpret_cast<const float4*>(C + tok * D + k))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     };
     load(0);
@@ -263,14 +273,15 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
       for (int i = 0; i < 8; ++i) {
         const int f = t + 128 * i;
         const int row = f >> 3, c = f & 7;
-        float4 h, l;
-        split_tf32(buf[i].x, h.x, l.x);
-        split_tf32(buf[i].y, h.y, l.y);
-        split_tf32(buf[i].z, h.z, l.z);
-        split_tf32(buf[i].w, h.w, l.w);
         const uint32_t off = swz_off(row, c);
-        *reinterpret_cast<float4*>(hi + off) = h;
-        *reinterpret_cast<float4*>(lo + off) = l;
+        const float4 x0 = buf[2 * i], x1 = buf[2 * i + 1];
+        uint32_t h[4], l[4];
+        split_bf16x2(x0.x, x0.y, h[0], l[0]);
+        split_bf16x2(x0.z, x0.w, h[1], l[1]);
+        split_bf16x2(x1.x, x1.y, h[2], l[2]);
+        split_bf16x2(x1.z, x1.w, h[3], l[3]);
+        *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
       }
       fence_proxy_async();  // generic-proxy stores -> visible to the tensor cores
       mbar_arrive(&full[s]);
@@ -279,7 +290,7 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   } else if (warp == 4) {
     // ---- MMA issue (one thread)
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_tf32<kTcBM, BN>();
+      constexpr uint32_t idesc = idesc_bf16<kTcBM, BN>();
       for (int kt = 0; kt < nkt; ++kt) {
         const int s = kt % kTcStages;
         const uint32_t ph = (kt / kTcStages) & 1;
@@ -292,8 +303,8 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
 #pragma unroll
         for (int pass = 0; pass < 3; ++pass)
 #pragma unroll
-          for (int ks = 0; ks < kTcBK / 8; ++ks)  // K = 8 tf32 (32 bytes) per MMA
-            umma_tf32(tmem, smem_desc(pa[pass] + 32 * ks), smem_desc(pb[pass] + 32 * ks), idesc,
+          for (int ks = 0; ks < 4; ++ks)  // K = 16 bf16 (32 bytes) per MMA
+            umma_bf16(tmem, smem_desc(pa[pass] + 32 * ks), smem_desc(pb[pass] + 32 * ks), idesc,
                       (kt | pass | ks) != 0);
         umma_commit(&empty[s]);  // the stage is free once these MMAs are done
       }
@@ -421,7 +432,7 @@ template <int BN>
 cudaError_t launch_tc(const float* C, int64_t T, int D, int H, const float* W1, const float* W2,
                       const float* W3, unsigned char* Wp, float4* zpart, unsigned int* status,
                       cudaStream_t stream) {
-  const int nkt = (D + kTcBK - 1) / kTcBK;
+  const int nkt = (D + kTcKE - 1) / kTcKE;
   const int nhb = H / (BN / 2);
   prepack_weights_kernel<BN><<<dim3(nkt, nhb), 256, 0, stream>>>(W1, W2, D, H, nkt, Wp);
   cudaError_t err = cudaGetLastError();
@@ -441,7 +452,7 @@ cudaError_t launch_tc(const float* C, int64_t T, int D, int H, const float* W1, 
 size_t route_workspace_bytes(int64_t T, int D, int H) {
   const int BN = H >= 128 ? 256 : 128;
   const int nhb = H / (BN / 2);
-  const int nkt = (D + kTcBK - 1) / kTcBK;
+  const int nkt = (D + kTcKE - 1) / kTcKE;
   const size_t wp = (size_t)nhb * nkt * 2 * BN * 128;
   return (size_t)align128(wp) + (size_t)align128((uint64_t)T * nhb * 16) + 1024;
 }
@@ -452,7 +463,7 @@ cudaError_t launch_router_tc(const float* C, int64_t T, int D, int H, const floa
                              int* nhb_out) {
   const int BN = H >= 128 ? 256 : 128;
   const int nhb = H / (BN / 2);
-  const int nkt = (D + kTcBK - 1) / kTcBK;
+  const int nkt = (D + kTcKE - 1) / kTcKE;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   unsigned char* Wp = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(ws) + 1023) & ~uintptr_t(1023));

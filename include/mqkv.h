@@ -260,9 +260,13 @@ mq_status mq_device_status(uint32_t* h_flags, int32_t clear, void* stream);
  *                h_seq_lens, D, H) bytes (weights split for the tensor
  *                cores, partial scores); contents on entry are ignored
  * Constraints: 1 <= D, D % 4 == 0; H in {64, 128, 256}.
- * The two projections run on the tensor cores in three tf32 passes
- * (hi*hi + hi*lo + lo*hi of a tf32 high part and an fp32 remainder), which
- * keeps each product within about 2^-21 relative of fp32.
+ * The two projections run on the tensor cores in three bf16 passes
+ * (hi*hi + hi*lo + lo*hi of a bf16 high part and the bf16 of the remainder,
+ * fp32 accumulation), which keeps each product within about 2^-16 relative;
+ * the scores agree with exact arithmetic to about 1e-4 relative, well inside
+ * the gap a routing decision needs before rounding can flip it (a token's
+ * choice can only change when its two best scores are within twice the
+ * error).
  * ------------------------------------------------------------------------- */
 size_t mq_route_workspace_bytes(const mq_shape* shape, const int32_t* h_seq_lens,
                                 int32_t D, int32_t H);
