@@ -18,8 +18,9 @@ NEAR_TIE = 1e-3
 # Score error allowed against the fp64 oracle.  A token's argmax can change
 # only if some score moves by half its top-2 gap or more, so any error below
 # NEAR_TIE / 2 keeps every choice outside the near-tie band exact.  The
-# tensor-core accumulator truncates once per MMA (about D/8 * 2^-24 relative),
-# which reaches ~1.5e-4 at D = 5120; 4e-4 keeps a margin under NEAR_TIE / 2.
+# router's three bf16 passes (~2^-16 relative per product, fp32 tensor-core
+# accumulation) measure up to ~8e-5 at D = 5120; 4e-4 keeps a margin under
+# NEAR_TIE / 2.
 SCORE_TOL = 4e-4
 
 
