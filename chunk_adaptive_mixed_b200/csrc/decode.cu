@@ -543,25 +543,42 @@ decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
   float M = -INFINITY, l = 0.f, acc[PER_LANE];
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) acc[i] = 0.f;
-  for (int it = i0 + warp; it < i1; it += NW) {
-    const int64_t wi = ((int64_t)it * Hkv + g) * QPG + hh;
-    const float2 ml = ws_ml[wi];
-    const float* a = ws_acc + wi * D + lane * PER_LANE;
-    float v[PER_LANE];
-    if constexpr (PER_LANE == 4) {
-      const float4 t = *reinterpret_cast<const float4*>(a);
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-    } else {
-      const float2 t = *reinterpret_cast<const float2*>(a);
-      v[0] = t.x; v[1] = t.y;
-    }
-    const float Mn = fmaxf(M, ml.x);
-    const float fa = M == -INFINITY ? 0.f : exp2f(M - Mn);
-    const float fb = ml.x == -INFINITY ? 0.f : exp2f(ml.x - Mn);
-    l = l * fa + ml.y * fb;
+  // kU items per round, all loaded before any is merged (independent loads
+  // in flight instead of one dependent load at a time)
+  constexpr int kU = 4;
+  for (int it0 = i0 + warp; it0 < i1; it0 += NW * kU) {
+    float2 ml[kU];
+    float v[kU][PER_LANE];
 #pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) acc[i] = acc[i] * fa + v[i] * fb;
-    M = Mn;
+    for (int u = 0; u < kU; ++u) {
+      const int it = it0 + u * NW;
+      ml[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int i = 0; i < PER_LANE; ++i) v[u][i] = 0.f;
+      if (it < i1) {
+        const int64_t wi = ((int64_t)it * Hkv + g) * QPG + hh;
+        ml[u] = ws_ml[wi];
+        const float* a = ws_acc + wi * D + lane * PER_LANE;
+        if constexpr (PER_LANE == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(a);
+          v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(a);
+          v[u][0] = t.x; v[u][1] = t.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (ml[u].x == -INFINITY) continue;  // past the end, or an item with no tokens
+      const float Mn = fmaxf(M, ml[u].x);
+      const float fa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      const float fb = exp2f(ml[u].x - Mn);
+      l = l * fa + ml[u].y * fb;
+#pragma unroll
+      for (int i = 0; i < PER_LANE; ++i) acc[i] = acc[i] * fa + v[u][i] * fb;
+      M = Mn;
+    }
   }
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) s_acc[warp][lane * PER_LANE + i] = acc[i];
