@@ -272,6 +272,47 @@ def test_pack_adversarial_values_bit_exact(dtype):
             raise AssertionError(f"{mapname}: {len(bad)} packed bytes differ, first at {bad[:8]}")
 
 
+def _tie_groups(n_groups, bits, rng):
+    """fp16 groups whose range is (2^b - 1) * m * 2^e (m odd, small): many
+    values sit exactly on, or one fp16 step beside, the half-integer points
+    min + (k + 1/2) s, at scales of every binade."""
+    lev = 2 ** bits - 1
+    g = np.empty((n_groups, 32), np.float32)
+    for i in range(n_groups):
+        mn = np.float16(rng.uniform(-50, 50) * 2.0 ** rng.integers(-12, 3))
+        d = lev * (1 + 2 * rng.integers(0, 8)) * 2.0 ** float(rng.integers(-14, 6))
+        mx = np.float16(np.float32(mn) + np.float32(d))
+        s = (np.float32(mx) - np.float32(mn)) / np.float32(lev)
+        pts = np.float32(mn) + (rng.integers(0, lev, 32) + np.float32(0.5)) * s
+        x = pts.astype(np.float16)
+        step = rng.integers(-1, 2, 32)                  # one fp16 step off, or on the point
+        x = np.where(step < 0, np.nextafter(x, np.float16(-np.inf)),
+                     np.where(step > 0, np.nextafter(x, np.float16(np.inf)), x))
+        x = np.clip(x, mn, mx).astype(np.float32)
+        x[0], x[1] = np.float32(mn), np.float32(mx)
+        g[i] = x
+    return g
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_pack_fp16_half_integer_quotients_bit_exact(bits):
+    # the fp16 encoder derives RN(t / s) without a division; these groups put
+    # the quotient on, or a rounding step beside, k + 1/2 at many scales
+    case = Case(np.array([256, 96], np.int32), 4, 4, 128, 32, "f16")
+    rng = np.random.default_rng(100 + bits)
+    n = case.T * case.Hkv * case.d // 32
+    K = _tie_groups(n, bits, rng).reshape(case.T, case.Hkv, case.d)
+    V = _tie_groups(n, bits, rng).reshape(case.T, case.Hkv, case.d)
+    Kt, Vt = torch.from_numpy(K).half(), torch.from_numpy(V).half()
+    cmap = np.full(int(W.num_chunks(case.lens, case.L).sum()), 1 if bits == 4 else 2, np.uint8)
+    layout = gpu_layout(case, cmap)
+    packed, pb = gpu_pack(case, layout, Kt.to(dev()), Vt.to(dev()))
+    ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, Kt.numpy(), Vt.numpy())
+    got = packed[:pb].cpu().numpy()
+    bad = np.nonzero(got != ref)[0]
+    assert len(bad) == 0, f"{len(bad)} packed bytes differ, first at {bad[:8]}"
+
+
 @pytest.mark.parametrize("hq,hkv", [(8, 2), (4, 4)])
 def test_decode_with_very_large_groups(hq, hkv):
     # groups whose range reaches ~6e4 (scale ~4e4 at INT2): products of softmax
