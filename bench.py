@@ -81,8 +81,8 @@ def measured_peaks():
 # profiles/), valid only for the pack kernel source (pack.cu) with this
 # SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "7742da4223f6323a87c63055c1133fcdf114037ed7413ea3c5cf0283c07bb5e3",
-                "bytes_per_launch": 2155172608 + 856218112}
+                "sha256": "a165b88fd0b8f3200666333218a3e71550ec847e070838b0539a073d89b871bd",
+                "bytes_per_launch": 2147894016 + 845130240}
 
 
 def pack_sources_sha256():
