@@ -21,8 +21,8 @@
 // instruction reads whole sectors.  Per tile:
 //   lanes: LPT lanes cover one token (SL dims each), TPW tokens per tile; the
 //          lane keeps its SL query values of all Hq/Hkv heads in registers
-//   scores: q . code on the raw codes (expanded with one byte-permute and a
-//          mask per value pair, see spread_byte), dequantisation folded in per
+//   scores: q . code on the raw codes (one mask per code, see code_bits),
+//          dequantisation folded in per
 //          group: q . khat = s * (q . code) + min * sum(q); shuffle-reduced
 //          over the token's LPT lanes
 //   softmax: online, log2 domain, with a lazily moved reference maximum
@@ -48,7 +48,7 @@ template <int D, int QPG, int E>
 struct Geo {
   static constexpr int BITS = E == 0 ? 16 : (E == 1 ? 4 : 2);
   static constexpr int SL_INT = 32 / QPG;
-  static constexpr int SL = E == 0 ? (SL_INT < 8 ? SL_INT : 8) : SL_INT;
+  static constexpr int SL = E == 0 ? (SL_INT < 16 ? SL_INT : 16) : SL_INT;
   static constexpr int LPT = D / SL;
   static constexpr int TPW = 32 / LPT;
   static constexpr int PIECE = SL * BITS / 8;   // code bytes of one lane's slice
@@ -107,28 +107,44 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Code extraction without shifts.  __byte_perm puts byte m of a code word
-// into bytes 2 and 1 of a word whose byte 3 is 0x43 (the exponent of 2^7):
-//   [0x43 | B | B | 0].
-// Masking keeps one code in the mantissa, giving exactly 128 + c * 2^k:
-//   INT4: low nibble  & 0xFF0F0000 -> 128 + c        (k = 0)
-//         high nibble & 0xFF00F000 -> 128 + c / 16   (k = -4, from byte 1)
-//   INT2: & 0xFF030000 -> 128 + c, & 0xFF0C0000 -> 128 + 4c,
-//         & 0xFF300000 -> 128 + 16c, & 0xFF00C000 -> 128 + c / 4.
-// (Byte 2's top bit is the exponent's lowest bit, so the code in that
-// position is read from the byte-1 copy instead.)  Each value has at most 12
-// significant bits, so its product with an fp16 query (11 bits), pre-scaled
-// by 2^-k, is exact in fp32.
-__device__ __forceinline__ uint32_t spread_byte(uint32_t word, int m) {
-  return __byte_perm(word, 0x43u, 0x4005u | ((uint32_t)m << 8) | ((uint32_t)m << 4));
+// Code extraction by masking in place.  A 32-bit pattern below 2^24, read as
+// an fp32 number, is exactly pattern * 2^-149 (a subnormal, or exponent field
+// 1 where the spacing is the same), so masking one code of a packed word
+// leaves the float c * 2^(o - 149), o the code's bit offset; codes at offsets
+// 24 and up are first moved down one byte (offset o - 8).  The f32x2 FMAs
+// take subnormal operands without flushing (no .ftz), and the factor that
+// multiplies a code carries the compensating power of two:
+//   scores: query pre-scaled by 2^(kQExp - o), product q c 2^(kQExp - 149)
+//   values: weight scaled by 2^kWExp; the accumulator of position o holds
+//           sum p s c 2^(kWExp - 149 + o) and is rescaled at the end.
+// A code has at most 4 significant bits and an fp16 query 11, so each score
+// product is exact in fp32 (above the subnormal range, |q| >= 2^-41), and no
+// offset is subtracted afterwards.  Bounds: |q| < 2^64 keeps the scaled
+// query finite; weights stay below 2^8 (lazy rescaling) and s below 2^16, so
+// the scaled weight stays below 2^124.
+constexpr int kQExp = 64;
+constexpr int kWExp = 100;
+
+__device__ __forceinline__ constexpr float pow2f(int e) {
+  float r = 1.0f;
+  for (int i = 0; i < e; ++i) r *= 2.0f;
+  for (int i = 0; i > e; --i) r *= 0.5f;
+  return r;
 }
 
-// Per-position scale 2^-k of the code values above (query pre-scaling), and
-// its inverse (applied to value accumulators at the end).
+// Bit offset of code v of a lane's slice after code_bits.
 template <int BITS>
-__device__ __forceinline__ constexpr float pos_scale(int i) {
-  if constexpr (BITS == 4) return i % 2 == 0 ? 1.0f : 16.0f;
-  else return (i % 4) == 0 ? 1.0f : ((i % 4) == 1 ? 0.25f : ((i % 4) == 2 ? 0.0625f : 4.0f));
+__device__ __forceinline__ constexpr int code_off(int v) {
+  return (v * BITS) % 32 + BITS <= 24 ? (v * BITS) % 32 : (v * BITS) % 32 - 8;
+}
+
+// Code v of a lane's slice (words LSB-first), in place: c << code_off(v).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_bits(const uint32_t* words, int v) {
+  constexpr uint32_t m = (1u << BITS) - 1u;
+  const uint32_t w = words[(v * BITS) / 32];
+  const int o = (v * BITS) % 32;
+  return o + BITS <= 24 ? (w & (m << o)) : ((w >> 8) & (m << (o - 8)));
 }
 
 // One lane's copy units of one iteration: 16-byte pieces of the iteration's
@@ -194,14 +210,14 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
   const int tl = lane / LPT, sl = lane % LPT;
   const int iters = (n + TPW - 1) / TPW;
 
-  CopyPlan<STRIDE> cp;
-  plan_copies<Gm, STRIDE>(cp, regk, regv, soff, t0);
+  CopyPlan<Gm::STAGE> cp;  // this precision's units (the ring stride fits the largest)
+  plan_copies<Gm, Gm::STAGE>(cp, regk, regv, soff, t0);
   auto issue = [&](int it) {
     if (it < iters) {
       const int nv = min(TPW, n - it * TPW);
       unsigned char* st = ring + (it % kRing) * STRIDE;
 #pragma unroll
-      for (int i = 0; i < CopyPlan<STRIDE>::U; ++i)
+      for (int i = 0; i < CopyPlan<Gm::STAGE>::U; ++i)
         if (cp.used[i] && cp.row[i] < nv)
           cp_async16(st + cp.dst[i], cp.src[i] + (uint64_t)it * cp.step[i]);
     }
@@ -212,12 +228,11 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
 
   // ---- query slice of every head, in value pairs, pre-scaled per code position
   uint64_t qp[QPG][NP];
-  float qs[QPG], qb[QPG];
+  float qs[QPG];
 #pragma unroll
   for (int h = 0; h < QPG; ++h) {
     const int64_t base = qbase + (int64_t)h * D + sl * SL;
     qs[h] = 0.f;
-    qb[h] = 0.f;
 #pragma unroll
     for (int j = 0; j < SL; j += 2) {
       float a, b;
@@ -232,13 +247,11 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
       }
       qs[h] += a + b;
       if constexpr (E != 0) {
-        a *= pos_scale<BITS>(j);
-        b *= pos_scale<BITS>(j + 1);
-        qb[h] += a + b;
+        a *= pow2f(kQExp - code_off<BITS>(j));
+        b *= pow2f(kQExp - code_off<BITS>(j + 1));
       }
       qp[h][j / 2] = pk2(a, b);
     }
-    qb[h] *= 128.0f;
   }
 
   uint64_t acc[QPG][NP];
@@ -251,7 +264,6 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
 #pragma unroll
     for (int j = 0; j < NP; ++j) acc[h][j] = 0ull;
   }
-  const uint64_t k128 = pk2(128.0f, 128.0f);
   const int grp = (sl * SL) / kGroup;
 
   for (int it = 0; it < iters; ++it) {
@@ -268,7 +280,7 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
           *reinterpret_cast<const uint32_t*>(st + 2 * Gm::CODES + tl * Gm::SROW + grp * 4));
       const float2 b = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(
           st + 2 * Gm::CODES + Gm::SCALES + tl * Gm::SROW + grp * 4));
-      ks = a.x; km = a.y; vs = b.x; vm = b.y;
+      ks = a.x * pow2f(149 - kQExp); km = a.y; vs = b.x * pow2f(kWExp); vm = b.y;
     }
     // ---- scores: q . code (pairs) in kChains independent accumulator chains
     // (short dependency chains), then the group's scale and min
@@ -299,23 +311,10 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
         words[0] = BYTES == 2 ? *reinterpret_cast<const unsigned short*>(kp) : *kp;
       }
 #pragma unroll
-      for (int mb = 0; mb < BYTES; ++mb) {
-        const uint32_t t = spread_byte(words[mb / 4], mb % 4);
-        if constexpr (BITS == 4) {
-          const uint64_t x = pk2u(t & 0xFF0F0000u, t & 0xFF00F000u);
+      for (int i = 0; i < NP; ++i) {
+        const uint64_t x = pk2u(code_bits<BITS>(words, 2 * i), code_bits<BITS>(words, 2 * i + 1));
 #pragma unroll
-          for (int h = 0; h < QPG; ++h)
-            dot2[h][mb % kChains] = fma2(x, qp[h][mb], dot2[h][mb % kChains]);
-        } else {
-          const uint64_t x0 = pk2u(t & 0xFF030000u, t & 0xFF0C0000u);
-          const uint64_t x1 = pk2u(t & 0xFF300000u, t & 0xFF00C000u);
-#pragma unroll
-          for (int h = 0; h < QPG; ++h) {
-            dot2[h][(2 * mb) % kChains] = fma2(x0, qp[h][2 * mb], dot2[h][(2 * mb) % kChains]);
-            dot2[h][(2 * mb + 1) % kChains] =
-                fma2(x1, qp[h][2 * mb + 1], dot2[h][(2 * mb + 1) % kChains]);
-          }
-        }
+        for (int h = 0; h < QPG; ++h) dot2[h][i % kChains] = fma2(x, qp[h][i], dot2[h][i % kChains]);
       }
     }
     float part[QPG];
@@ -324,7 +323,7 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
       float dot = 0.f;
 #pragma unroll
       for (int c = 0; c < kChains; ++c) dot += lo2(dot2[h][c]) + hi2(dot2[h][c]);
-      part[h] = E == 0 ? dot : fmaf(ks, dot - qb[h], km * qs[h]);
+      part[h] = E == 0 ? dot : fmaf(ks, dot, km * qs[h]);
     }
 #pragma unroll
     for (int off = 1; off < LPT; off <<= 1)
@@ -378,21 +377,10 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
           words[0] = BYTES == 2 ? *reinterpret_cast<const unsigned short*>(vp) : *vp;
         }
 #pragma unroll
-        for (int mb = 0; mb < BYTES; ++mb) {
-          const uint32_t t = spread_byte(words[mb / 4], mb % 4);
-          if constexpr (BITS == 4) {
-            const uint64_t x = sub2(pk2u(t & 0xFF0F0000u, t & 0xFF00F000u), k128);
+        for (int i = 0; i < NP; ++i) {
+          const uint64_t x = pk2u(code_bits<BITS>(words, 2 * i), code_bits<BITS>(words, 2 * i + 1));
 #pragma unroll
-            for (int h = 0; h < QPG; ++h) acc[h][mb] = fma2(x, w2[h], acc[h][mb]);
-          } else {
-            const uint64_t x0 = sub2(pk2u(t & 0xFF030000u, t & 0xFF0C0000u), k128);
-            const uint64_t x1 = sub2(pk2u(t & 0xFF300000u, t & 0xFF00C000u), k128);
-#pragma unroll
-            for (int h = 0; h < QPG; ++h) {
-              acc[h][2 * mb] = fma2(x0, w2[h], acc[h][2 * mb]);
-              acc[h][2 * mb + 1] = fma2(x1, w2[h], acc[h][2 * mb + 1]);
-            }
-          }
+          for (int h = 0; h < QPG; ++h) acc[h][i] = fma2(x, w2[h], acc[h][i]);
         }
       }
     }
@@ -406,8 +394,9 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
   for (int h = 0; h < QPG; ++h)
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-      av[h][2 * j] = lo2(acc[h][j]) * (E == 0 ? 1.f : pos_scale<BITS>(2 * j));
-      av[h][2 * j + 1] = hi2(acc[h][j]) * (E == 0 ? 1.f : pos_scale<BITS>(2 * j + 1));
+      av[h][2 * j] = lo2(acc[h][j]) * (E == 0 ? 1.f : pow2f(149 - kWExp - code_off<BITS>(2 * j)));
+      av[h][2 * j + 1] =
+          hi2(acc[h][j]) * (E == 0 ? 1.f : pow2f(149 - kWExp - code_off<BITS>(2 * j + 1)));
     }
 #pragma unroll
   for (int off = LPT; off < 32; off <<= 1) {
