@@ -101,6 +101,18 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// 2^x by the hardware approximation (max error 2 ulp), results below 2^-126
+// flushed to zero: softmax weights that small do not register in the sums.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -255,11 +267,12 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
   }
 
   uint64_t acc[QPG][NP];
-  float bias[QPG], m[QPG], l[QPG];
+  float bias[QPG], m[QPG], m8[QPG], l[QPG];  // m8 = m + kRescale
 #pragma unroll
   for (int h = 0; h < QPG; ++h) {
     bias[h] = 0.f;
     m[h] = -INFINITY;
+    m8[h] = -INFINITY;
     l[h] = 0.f;
 #pragma unroll
     for (int j = 0; j < NP; ++j) acc[h][j] = 0ull;
@@ -320,9 +333,14 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
     float part[QPG];
 #pragma unroll
     for (int h = 0; h < QPG; ++h) {
-      float dot = 0.f;
+      uint64_t d2 = dot2[h][0];
+      if constexpr (kChains == 4) {
+        d2 = add2(add2(dot2[h][0], dot2[h][1]), add2(dot2[h][2], dot2[h][3]));
+      } else {
 #pragma unroll
-      for (int c = 0; c < kChains; ++c) dot += lo2(dot2[h][c]) + hi2(dot2[h][c]);
+        for (int c = 1; c < kChains; ++c) d2 = add2(d2, dot2[h][c]);
+      }
+      const float dot = lo2(d2) + hi2(d2);
       part[h] = E == 0 ? dot : fmaf(ks, dot, km * qs[h]);
     }
 #pragma unroll
@@ -336,27 +354,32 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
       // lazy rescaling: the reference maximum moves only when a score exceeds
       // it by more than kRescale (log2 units), so weights stay below
       // 2^kRescale; (m, l, acc) remain consistent for any reference
-      if (sc > m[h] + kRescale) {
-        const float a = exp2f(m[h] - sc);
+      // (m8 is kept only with one query head per kv-head: with several, the
+      // registers are better spent elsewhere)
+      if (sc > (QPG == 1 ? m8[h] : m[h] + kRescale)) {
+        const float a = ex2_ftz(m[h] - sc);
         const uint64_t a2 = pk2(a, a);
         l[h] *= a;
         bias[h] *= a;
 #pragma unroll
         for (int j = 0; j < NP; ++j) acc[h][j] = fma2(acc[h][j], a2, 0ull);
         m[h] = sc;
+        if constexpr (QPG == 1) m8[h] = sc + kRescale;
       }
-      p[h] = valid ? exp2f(sc - m[h]) : 0.f;
+      p[h] = valid ? ex2_ftz(sc - m[h]) : 0.f;
       l[h] += p[h];
     }
-    // ---- values (lanes past the item's last token hold stale stage bytes,
-    // which may decode to NaN: they skip the accumulation instead)
-    if (valid) {
+    // ---- values.  Lanes past the item's last token hold stale stage bytes:
+    // their fp16 values and scales may be NaN, so FP16 tiles skip the
+    // accumulation and quantised tiles zero the weight by a select (masked
+    // codes are always finite, so they then add exactly 0).
+    if (E != 0 || valid) {
       uint64_t w2[QPG];
 #pragma unroll
       for (int h = 0; h < QPG; ++h) {
-        const float wgt = E == 0 ? p[h] : p[h] * vs;
+        const float wgt = E == 0 ? p[h] : (valid ? p[h] * vs : 0.f);
         w2[h] = pk2(wgt, wgt);
-        if constexpr (E != 0) bias[h] = fmaf(p[h], vm, bias[h]);
+        if constexpr (E != 0) bias[h] = valid ? fmaf(p[h], vm, bias[h]) : bias[h];
       }
       if constexpr (E == 0) {
         const uint32_t* wv = reinterpret_cast<const uint32_t*>(vp);
