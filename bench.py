@@ -81,8 +81,8 @@ def measured_peaks():
 # profiles/), valid only for the pack kernel source (pack.cu) with this
 # SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "a165b88fd0b8f3200666333218a3e71550ec847e070838b0539a073d89b871bd",
-                "bytes_per_launch": 2147894016 + 845130240}
+                "sha256": "54f519c0da85c9212875d6fe6568176589515438e04963f0a80a3e65e745f14c",
+                "bytes_per_launch": 2148346368 + 843314688}
 
 
 def pack_sources_sha256():
