@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "decode attn tokens/s & packed-KV HBM GB/s (% of B200 peak); pack GB/s"
 DEFAULT_WORKLOAD = "llama2_7b_32l"
 L2_BYTES = 126 * 2 ** 20
+SPEC_HBM_GBS = 8000.0   # B200 HBM3e data-sheet bandwidth (context beside the measured peak)
 
 
 def parse():
@@ -547,33 +548,65 @@ def run_ours(args, rank, world, local_rank):
         pb = int(np.mean([M.mq_packed_bytes(S.layout_of(l)) for l in range(w.layers)]))
     mix = np.bincount(S.chunk_expert[:S.N].cpu().numpy(), minlength=3) / max(S.N, 1)
 
-    # per-kernel events for every pack launch and the first decode step
+    # per-kernel events for every pack launch and the first decode step.
+    # Workloads whose K/V fit twice in L2 would leave the next step's inputs
+    # cached: those write a 2 x L2 buffer before every step, outside the
+    # step's events, and report the unflushed time beside it.
     E = torch.cuda.Event
-    timers_all = []
+    flush = S.kv_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device) if flush else None
+
+    def timed_steps(with_flush):
+        timers, spans = [], []
+        for _ in range(args.steps):
+            if with_flush:
+                flush_buf.fill_(1)
+            tm = {"route": (E(enable_timing=True), E(enable_timing=True)),
+                  "pack": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)],
+                  "decode": [(E(enable_timing=True), E(enable_timing=True))
+                             for _ in range(w.layers)]}
+            if with_flush or not spans:
+                spans.append((E(enable_timing=True), E(enable_timing=True)))
+                spans[-1][0].record()
+            S.step(tm)
+            if with_flush:
+                spans[-1][1].record()
+            timers.append(tm)
+        if not with_flush:
+            spans[-1][1].record()
+        return timers, spans
+
+    no_flush = None
+    if flush:
+        barrier()
+        torch.cuda.synchronize()
+        _, spans_nf = timed_steps(False)
+        torch.cuda.synchronize()
+        ms_nf = reduce_timing(sum(a.elapsed_time(b) for a, b in spans_nf), device)
+        no_flush = {"ms_per_step": ms_nf / args.steps,
+                    "value": job_throughput(S.B * w.decode_steps, world, ms_nf / args.steps)
+                    if not args.context_split else S.B * w.decode_steps / (ms_nf / args.steps / 1e3)}
     barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank)
     sampler.start()
-    t_start, t_end = E(enable_timing=True), E(enable_timing=True)
-    t_start.record()
-    for _ in range(args.steps):
-        tm = {"route": (E(enable_timing=True), E(enable_timing=True)),
-              "pack": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)],
-              "decode": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)]}
-        S.step(tm)
-        timers_all.append(tm)
-    t_end.record()
+    timers_all, spans = timed_steps(flush)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     assert M.mq_device_status() == 0, "device-side check failed in the timed region"
-    ms = reduce_timing(t_start.elapsed_time(t_end), device)
+    ms = reduce_timing(sum(a.elapsed_time(b) for a, b in spans), device)
     ms_step = ms / args.steps
     pack_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["pack"]]
     dec_ms = [a.elapsed_time(b) for tm in timers_all for a, b in tm["decode"]]
     route_ms = float(np.mean([tm["route"][0].elapsed_time(tm["route"][1]) for tm in timers_all]))
     pack_avg = float(np.mean(pack_ms))
     dec_avg = float(np.mean(dec_ms))
+
+    def spread(xs):
+        """Median, 10th and 90th percentile of per-launch times (ms)."""
+        return {"median_ms": float(np.median(xs)), "p10_ms": float(np.percentile(xs, 10)),
+                "p90_ms": float(np.percentile(xs, 90)), "launches": len(xs)}
 
     tokens_per_step = S.B * w.decode_steps
     if args.context_split:
@@ -612,8 +645,9 @@ def run_ours(args, rank, world, local_rank):
                        "parallelism": (f"cp{world} (context split, records all-gathered)"
                                        if args.context_split
                                        else f"dp{world} (independent batches)"),
-                       "l2": "inputs larger than L2 (no flush needed)" if S.kv_bytes > L2_BYTES
-                       else "inputs fit in L2"},
+                       "l2": ("2 x L2 buffer written before every step (outside its events); "
+                              "unflushed time in no_flush") if flush
+                       else "inputs larger than 2 x L2 (no flush needed)"},
             "roofline": {"bound": "hbm", "kernel": "pack_kernel",
                          "achieved": pack_gbs, "peak": peak, "unit": "GB/s",
                          "frac": pack_gbs / peak, "traffic": pack_traffic(w, S, seed),
@@ -621,10 +655,13 @@ def run_ours(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": pack_bytes,
                          "avg_launch_ms": pack_avg},
             "decode_attn": {"GB/s": dec_gbs, "frac": dec_gbs / peak, "avg_ms_per_layer": dec_avg,
+                            "frac_of_spec": dec_gbs / SPEC_HBM_GBS,
                             "tokens_per_s_attention_only": S.B / (dec_avg * w.layers / 1e3),
-                            "algorithmic_bytes_per_layer": dec_bytes},
+                            "algorithmic_bytes_per_layer": dec_bytes, **spread(dec_ms)},
             "route": route_summary(S, route_ms, peaks_all()),
-            "pack": {"GB/s": pack_gbs, "frac": pack_gbs / peak, "avg_ms_per_layer": pack_avg},
+            "pack": {"GB/s": pack_gbs, "frac": pack_gbs / peak, "avg_ms_per_layer": pack_avg,
+                     "frac_of_spec": pack_gbs / SPEC_HBM_GBS, **spread(pack_ms)},
+            "no_flush": no_flush,
             "packed_bytes_per_layer": pb,
             "chunk_mix": [round(float(x), 4) for x in mix],
             "avg_bits": float(np.dot(mix, [16, 4, 2])),

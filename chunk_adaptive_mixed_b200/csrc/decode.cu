@@ -668,11 +668,14 @@ combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ p
 //           products keep fp32-level accuracy, O held in units of a power
 //           of two raised with the largest scale seen so P' fits fp16; the
 //           mins enter as sum_t p_t min_t per group.
-// Codes become exact fp16 integers (one byte-permute, one mask and one fma
-// per pair).  The dims of a k-step are permuted identically in K and Q so
-// that each lane reads whole bytes: k = 2t, 2t+1, 2t+8, 2t+9 of k-step
-// (group g, half hh) are dims 32g + 8t + 4hh + {0, 1, 2, 3} (t = lane % 4).
-// V codes are expanded into a padded fp16 tile and fed to the MMA with
+// INT4 codes enter in place as fp16 c * 2^-24 (one shift and one mask per
+// pair, see nib_sub); INT2 codes become exact fp16 integers (one
+// byte-permute, one mask and one fma per pair).  The dims of a k-step are
+// permuted identically in K and Q so that each lane reads whole bytes:
+// k = 2t, 2t+1, 2t+8, 2t+9 of k-step (group g, half hh) are dims
+// 32g + 8t + 2hh + {0, 4, 1, 5} for INT4 and 32g + 8t + 4hh + {0, 1, 2, 3}
+// for INT2 (t = lane % 4).  V codes are expanded into a padded fp16 tile
+// (INT4 dims in nib_dim order inside each 8) and fed to the MMA with
 // ldmatrix.trans; FP16 segments feed K and V straight from the staged rows.
 // ============================================================================
 constexpr int kMmaWarps = 1;            // one worker warp per CTA: ~10 resident per SM
@@ -738,11 +741,17 @@ __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cas
 __device__ __forceinline__ uint32_t spread2(uint32_t w, int j) {
   return __byte_perm(w, 0x6464u, (uint32_t)j | 0x4000u | ((uint32_t)j << 8) | 0x0050u);
 }
-// INT4: byte j of w -> fp16 pair (low nibble, high nibble), exact
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, int j) {
-  const __half2 x = bits_h2(spread2(w, j) & 0xFFF0FF0Fu);   // (1024 + lo, 1024 + 16 hi)
-  return h2_bits(__hfma2(x, __floats2half2_rn(1.0f, 0.0625f), __floats2half2_rn(-1024.0f, -64.0f)));
+// INT4 in place: nibbles (i, i + 4) of w as an fp16 pair, each exactly
+// c * 2^-24 (an fp16 pattern below 0x0800 is pattern * 2^-24: subnormal, or
+// exponent field 1 with the same spacing).  No offset to remove; the 2^24
+// goes into the group scale (scores) or the output unit (values).
+__device__ __forceinline__ uint32_t nib_sub(uint32_t w, int i) {
+  return (w >> (4 * i)) & 0x000F000Fu;
 }
+// Dim order of the INT4 in-place pairs inside a word's 8 dims: slot p of
+// (nib_sub(w, 0), nib_sub(w, 1), nib_sub(w, 2), nib_sub(w, 3)) holds dim
+// nib_dim(p) = (p / 2) + 4 (p % 2).
+__device__ __forceinline__ constexpr int nib_dim(int p) { return (p >> 1) + 4 * (p & 1); }
 // INT2: byte j of w -> two fp16 pairs (c0, c1), (c2, c3), exact
 __device__ __forceinline__ void crumb_pairs(uint32_t w, int j, uint32_t& p01, uint32_t& p23) {
   const uint32_t x = spread2(w, j);
@@ -821,10 +830,19 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
     for (int g = 0; g < NG; ++g) part[g] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < NK; ++kk) {
-      const int d0 = E == 0 ? 16 * kk + 2 * tig : 32 * (kk / 2) + 8 * tig + 4 * (kk % 2);
-      const int d1 = E == 0 ? d0 + 8 : d0 + 2;
-      const uint32_t b0 = hv ? *reinterpret_cast<const uint32_t*>(qh + d0) : 0u;
-      const uint32_t b1 = hv ? *reinterpret_cast<const uint32_t*>(qh + d1) : 0u;
+      uint32_t b0, b1;
+      if constexpr (E == 1) {
+        // k = 2t, 2t+1 -> dims base + 2hh + {0, 4}; k = 2t+8, 2t+9 -> base + 2hh + {1, 5}
+        const int base = 32 * (kk / 2) + 8 * tig + 2 * (kk % 2);
+        const unsigned short* qs16 = reinterpret_cast<const unsigned short*>(qh);
+        b0 = hv ? (uint32_t)qs16[base] | ((uint32_t)qs16[base + 4] << 16) : 0u;
+        b1 = hv ? (uint32_t)qs16[base + 1] | ((uint32_t)qs16[base + 5] << 16) : 0u;
+      } else {
+        const int d0 = E == 0 ? 16 * kk + 2 * tig : 32 * (kk / 2) + 8 * tig + 4 * (kk % 2);
+        const int d1 = E == 0 ? d0 + 8 : d0 + 2;
+        b0 = hv ? *reinterpret_cast<const uint32_t*>(qh + d0) : 0u;
+        b1 = hv ? *reinterpret_cast<const uint32_t*>(qh + d1) : 0u;
+      }
       qb[kk][0] = b0;
       qb[kk][1] = b1;
       const float2 f0 = __half22float2(bits_h2(b0)), f1 = __half22float2(bits_h2(b1));
@@ -882,8 +900,8 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
           const uint32_t w1 = *reinterpret_cast<const uint32_t*>(st + G::KOFF + r1 * G::KROW + 4 * (4 * g + tig));
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh)
-            mma16816(acc, nib_pair(w0, 2 * hh), nib_pair(w1, 2 * hh), nib_pair(w0, 2 * hh + 1),
-                     nib_pair(w1, 2 * hh + 1), qb[2 * g + hh][0], qb[2 * g + hh][1]);
+            mma16816(acc, nib_sub(w0, 2 * hh), nib_sub(w1, 2 * hh), nib_sub(w0, 2 * hh + 1),
+                     nib_sub(w1, 2 * hh + 1), qb[2 * g + hh][0], qb[2 * g + hh][1]);
         } else {
           const uint32_t h0 = *reinterpret_cast<const unsigned short*>(st + G::KOFF + r0 * G::KROW + 8 * g + 2 * tig);
           const uint32_t h1 = *reinterpret_cast<const unsigned short*>(st + G::KOFF + r1 * G::KROW + 8 * g + 2 * tig);
@@ -895,8 +913,12 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
             mma16816(acc, a0, a1, a2, a3, qb[2 * g + hh][0], qb[2 * g + hh][1]);
           }
         }
-        const float2 sm0 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r0 * G::SROW + 4 * g));
-        const float2 sm1 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r1 * G::SROW + 4 * g));
+        float2 sm0 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r0 * G::SROW + 4 * g));
+        float2 sm1 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r1 * G::SROW + 4 * g));
+        if constexpr (E == 1) {  // codes entered as c * 2^-24
+          sm0.x *= 16777216.0f;
+          sm1.x *= 16777216.0f;
+        }
         s4[0] = fmaf(sm0.x, acc[0], fmaf(sm0.y, qsum[g][0], s4[0]));
         s4[1] = fmaf(sm0.x, acc[1], fmaf(sm0.y, qsum[g][1], s4[1]));
         s4[2] = fmaf(sm1.x, acc[2], fmaf(sm1.y, qsum[g][0], s4[2]));
@@ -951,9 +973,9 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
 #pragma unroll
         for (int k = 0; k < HB / 4; ++k) {
           const uint32_t wv = src[k];
-          if constexpr (E == 1) {
+          if constexpr (E == 1) {  // dims in nib_dim order, values c * 2^-24
             *reinterpret_cast<uint4*>(dst + 8 * k) =
-                make_uint4(nib_pair(wv, 0), nib_pair(wv, 1), nib_pair(wv, 2), nib_pair(wv, 3));
+                make_uint4(nib_sub(wv, 0), nib_sub(wv, 1), nib_sub(wv, 2), nib_sub(wv, 3));
           } else {
             uint32_t c[8];
 #pragma unroll
@@ -1057,14 +1079,18 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
     }
   }
 #pragma unroll
-  const float up = (E == 0 || abits == 0u) ? 1.f : __uint_as_float(abits);  // 2^A
+  // 2^A (and 2^24 for INT4 codes entered as c * 2^-24)
+  const float up = (E == 0 || abits == 0u) ? 1.f
+                   : __uint_as_float(abits) * (E == 1 ? 16777216.0f : 1.0f);
   for (int hj = 0; hj < 2; ++hj) {
     const int h = 2 * tig + hj;
     if (h < QPG) {
       float* dst = ws_acc + ((size_t)w * QPG + h) * D;
+      // row p of O^T is vbuf column p: dim p for FP16 / INT2, INT4 in nib_dim order
+      const int dg = E == 1 ? nib_dim(gid) : gid;
 #pragma unroll
       for (int mt = 0; mt < NK; ++mt) {
-        const int d0 = 16 * mt + gid, d1 = d0 + 8;
+        const int d0 = 16 * mt + dg, d1 = d0 + 8;
         dst[d0] = fmaf(o[mt][hj], up, vb[d0 / 32][hj]);
         dst[d1] = fmaf(o[mt][2 + hj], up, vb[d1 / 32][hj]);
       }
