@@ -11,7 +11,8 @@
 // within the tolerance the routing decisions allow, see include/mqkv.h).
 //
 // router_tc_kernel: one CTA owns 128 tokens and one block of HB hidden units
-// of both branches (an N = 2*HB accumulator in tensor memory).
+// of both branches (an N = 2*HB accumulator in tensor memory); the CTAs of
+// one token tile are consecutive in the grid.
 //   warps 0-3  load C (fp32) for the next k-tile, split it, store the two
 //              halves into 128B-swizzled K-major shared tiles, then run the
 //              epilogue: SiLU gate, W3 projection of this hidden block.
@@ -211,8 +212,10 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * kTcBM;
-  const int hb = blockIdx.y;
+  // the nhb hidden blocks of one token tile are adjacent CTAs, so they run
+  // together and all but the first read the tile's C rows from L2
+  const int64_t m0 = (int64_t)(blockIdx.x / nhb) * kTcBM;
+  const int hb = (int)(blockIdx.x % nhb);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
@@ -442,7 +445,7 @@ cudaError_t launch_tc(const float* C, int64_t T, int D, int H, const float* W1, 
   if ((err = cudaFuncSetAttribute(router_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess)
     return err;
-  const dim3 grid((unsigned)((T + kTcBM - 1) / kTcBM), (unsigned)nhb);
+  const dim3 grid((unsigned)(((T + kTcBM - 1) / kTcBM) * nhb));
   router_tc_kernel<BN><<<grid, kTcThreads, smem, stream>>>(C, T, D, nkt, Wp, W3, zpart, nhb, status);
   return cudaGetLastError();
 }
