@@ -691,10 +691,11 @@ combine_partials_kernel(int P, int64_t heads, int D, const float* __restrict__ p
 // (INT4 dims in nib_dim order inside each 8) and fed to the MMA with
 // ldmatrix.trans; FP16 segments feed K and V straight from the staged rows.
 // ============================================================================
-constexpr int kMmaWarps = 1;            // one worker warp per CTA: ~10 resident per SM
+constexpr int kMmaWarps = 1;            // one worker warp per CTA: 12 resident per SM
 constexpr int kMmaThreads = 32 * kMmaWarps;
 constexpr int kMmaTile = 16;            // tokens per tile
-constexpr int kMmaRing = 17408;         // bytes of one warp's copy ring (2 FP16 tiles at d=128)
+constexpr int kMmaRing = 17408;         // shared bytes of one warp: 2 FP16 tiles at d=128, or
+                                        // the quantised tiles' ring plus the V expansion tile
 constexpr int kRowPad = 16;             // bytes added to every staged code row
 
 template <int D, int E>
@@ -708,19 +709,23 @@ struct MG {
   static constexpr int KSOFF = 2 * kMmaTile * KROW;
   static constexpr int VSOFF = KSOFF + kMmaTile * SROW;
   static constexpr int STAGE = (VSOFF + kMmaTile * SROW + 15) / 16 * 16;
-  static constexpr int STAGES = kMmaRing / STAGE < 8 ? kMmaRing / STAGE : 8;
+  // quantised tiles leave the end of the warp's space to the V expansion tile
+  static constexpr int RING = E == 0 ? kMmaRing : kMmaRing - kMmaTile * (128 + 8) * 2;
+  static constexpr int STAGES = RING / STAGE < 8 ? RING / STAGE : 8;
   // 16-byte copy units of one tile: K codes, V codes, K scales, V scales
   static constexpr int CU = CROW / 16;                      // units per code row
   static constexpr int UNITS = 2 * kMmaTile * CU + 2 * SROW;  // a tile's scales: SROW units
 };
-static_assert(MG<128, 0>::STAGES >= 2 && MG<64, 0>::STAGES >= 2, "ring too small");
+static_assert(MG<128, 0>::STAGES >= 2 && MG<64, 0>::STAGES >= 2 && MG<128, 1>::STAGES >= 3 &&
+                  MG<128, 2>::STAGES >= 3,
+              "ring too small");
 
 constexpr int kVbufRow = 128 + 8;       // fp16 elements of one expanded V row (padded)
 constexpr int kVbufBytes = kMmaTile * kVbufRow * 2;
 
 template <int D>
 constexpr size_t mma_smem_bytes() {
-  return (size_t)kMmaWarps * (kMmaRing + kVbufBytes);
+  return (size_t)kMmaWarps * kMmaRing;
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -1114,7 +1119,7 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
 }
 
 template <int D, int QPG>
-__global__ void __launch_bounds__(kMmaThreads, 10)
+__global__ void __launch_bounds__(kMmaThreads, 12)
 decode_mma_kernel(const unsigned char* __restrict__ layout, const unsigned char* __restrict__ packed,
                   const __half* __restrict__ q, float scale_log2, float* __restrict__ ws_acc,
                   float2* __restrict__ ws_ml, unsigned int* __restrict__ counter,
@@ -1132,8 +1137,8 @@ decode_mma_kernel(const unsigned char* __restrict__ layout, const unsigned char*
     return;
   }
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  unsigned char* ring = smem_raw + (size_t)warp * (kMmaRing + kVbufBytes);
-  __half* vbuf = reinterpret_cast<__half*>(ring + kMmaRing);
+  unsigned char* ring = smem_raw + (size_t)warp * kMmaRing;
+  __half* vbuf = reinterpret_cast<__half*>(ring + kMmaRing - kVbufBytes);  // quantised tiles only
   for (;;) {
     unsigned int wi = 0;
     if (lane == 0) wi = atomicAdd(counter, 1u);
