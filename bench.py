@@ -82,8 +82,8 @@ def measured_peaks():
 # profiles/), valid only for the pack kernel source (pack.cu) with this
 # SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "54f519c0da85c9212875d6fe6568176589515438e04963f0a80a3e65e745f14c",
-                "bytes_per_launch": 2148346368 + 843314688}
+                "sha256": "a3a08a04cf53dd5d42e1fb6231e64fe083732404b654f9da30ac00c4e060144c",
+                "bytes_per_launch": 2148122624 + 843587328}
 
 
 def pack_sources_sha256():
