@@ -13,11 +13,12 @@
 // router_tc_kernel: one CTA owns 128 tokens and one block of HB hidden units
 // of both branches (an N = 2*HB accumulator in tensor memory); the CTAs of
 // one token tile are consecutive in the grid.
-//   warps 0-3  load C (fp32) for the next k-tile, split it, store the two
-//              halves into 128B-swizzled K-major shared tiles, then run the
+//   warps 0-7  load C (fp32) for the next k-tile, split it, store the two
+//              halves into 128B-swizzled K-major shared tiles (eight warps
+//              keep enough loads in flight); warps 0-3 then run the
 //              epilogue: SiLU gate, W3 projection of this hidden block.
-//   warp 4     allocates tensor memory and issues the MMAs (one thread).
-//   warp 5     brings the pre-split, pre-swizzled weight tiles with 1-D bulk
+//   warp 8     allocates tensor memory and issues the MMAs (one thread).
+//   warp 9     brings the pre-split, pre-swizzled weight tiles with 1-D bulk
 //              copies.
 // Two shared-memory stages; full/empty mbarriers; tcgen05.commit frees a
 // stage when its MMAs complete.  Every wait is bounded: on timeout the kernel
@@ -32,7 +33,11 @@ namespace {
 constexpr int kTcBM = 128;     // tokens per CTA (MMA M)
 constexpr int kTcKE = 64;      // bf16 k elements per k-tile (one 128-byte swizzle row)
 constexpr int kTcStages = 2;
-constexpr int kTcThreads = 192;
+constexpr int kTcProdWarps = 8;                  // producer warps (C split, epilogue)
+constexpr int kTcProd = 32 * kTcProdWarps;
+constexpr int kTcMmaWarp = kTcProdWarps;         // one thread issues the MMAs
+constexpr int kTcWeightWarp = kTcProdWarps + 1;  // one thread copies the weight tiles
+constexpr int kTcThreads = 32 * (kTcProdWarps + 2);
 constexpr uint32_t kTcWaitLimit = 1u << 24;
 
 // ---------------------------------------------------------------- PTX helpers
@@ -219,14 +224,14 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 128 + 1);
+      mbar_init(&full[s], kTcProd + 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == kTcMmaWarp) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
@@ -244,15 +249,16 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
     atomicExch(abort_flag, 1);
   };
 
-  if (warp < 4) {
+  if (warp < kTcProdWarps) {
     // ---- producers: C tile (128 rows x kTcKE fp32) -> split -> swizzled stores
-    const int t = threadIdx.x;  // 0..127
+    const int t = threadIdx.x;  // 0..kTcProd-1
     constexpr int NV = kTcKE / 32;  // float4 loads per 16-byte chunk of a part
-    float4 buf[8 * NV];
+    constexpr int PER = 8 * kTcBM / kTcProd;  // 16-byte chunks per thread and k-tile
+    float4 buf[PER * NV];
     auto load = [&](int kt) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int f = t + 128 * i;
+      for (int i = 0; i < PER; ++i) {
+        const int f = t + kTcProd * i;
         const int row = f >> 3, c = f & 7;
         const int64_t tok = m0 + row;
 #pragma unroll
@@ -273,8 +279,8 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
       unsigned char* hi = a_hi(s);
       unsigned char* lo = a_lo(s);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int f = t + 128 * i;
+      for (int i = 0; i < PER; ++i) {
+        const int f = t + kTcProd * i;
         const int row = f >> 3, c = f & 7;
         const uint32_t off = swz_off(row, c);
         const float4 x0 = buf[2 * i], x1 = buf[2 * i + 1];
@@ -290,7 +296,7 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
       mbar_arrive(&full[s]);
       if (kt + 1 < nkt) load(kt + 1);
     }
-  } else if (warp == 4) {
+  } else if (warp == kTcMmaWarp) {
     // ---- MMA issue (one thread)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16<kTcBM, BN>();
@@ -360,7 +366,7 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kTcMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, BN);
   }
