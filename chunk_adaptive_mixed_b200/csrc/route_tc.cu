@@ -254,8 +254,10 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
     const int t = threadIdx.x;  // 0..kTcProd-1
     constexpr int NV = kTcKE / 32;  // float4 loads per 16-byte chunk of a part
     constexpr int PER = 8 * kTcBM / kTcProd;  // 16-byte chunks per thread and k-tile
-    float4 buf[PER * NV];
-    auto load = [&](int kt) {
+    // two register buffers: the loads of k-tile kt + 2 are issued as soon as
+    // k-tile kt is stored, so two tiles of loads are in flight
+    float4 buf0[PER * NV], buf1[PER * NV];
+    auto load = [&](int kt, float4 (&buf)[PER * NV]) {
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int f = t + kTcProd * i;
@@ -270,12 +272,12 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
         }
       }
     };
-    load(0);
-    for (int kt = 0; kt < nkt; ++kt) {
+    // split k-tile kt into its stage; false when the kernel gives up
+    auto store = [&](int kt, const float4 (&buf)[PER * NV]) -> bool {
       const int s = kt % kTcStages;
       const uint32_t ph = (kt / kTcStages) & 1;
-      if (*(volatile int*)abort_flag) break;
-      if (!mbar_wait(&empty[s], ph ^ 1)) { fail(); break; }
+      if (*(volatile int*)abort_flag) return false;
+      if (!mbar_wait(&empty[s], ph ^ 1)) { fail(); return false; }
       unsigned char* hi = a_hi(s);
       unsigned char* lo = a_lo(s);
 #pragma unroll
@@ -294,7 +296,16 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
       }
       fence_proxy_async();  // generic-proxy stores -> visible to the tensor cores
       mbar_arrive(&full[s]);
-      if (kt + 1 < nkt) load(kt + 1);
+      return true;
+    };
+    load(0, buf0);
+    if (nkt > 1) load(1, buf1);
+    for (int kt = 0; kt < nkt; kt += 2) {
+      if (!store(kt, buf0)) break;
+      if (kt + 2 < nkt) load(kt + 2, buf0);
+      if (kt + 1 >= nkt) break;
+      if (!store(kt + 1, buf1)) break;
+      if (kt + 3 < nkt) load(kt + 3, buf1);
     }
   } else if (warp == kTcMmaWarp) {
     // ---- MMA issue (one thread)
