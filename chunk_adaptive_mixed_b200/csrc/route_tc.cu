@@ -15,8 +15,8 @@
 // one token tile are consecutive in the grid.
 //   warps 0-7  load C (fp32) for the next k-tile, split it, store the two
 //              halves into 128B-swizzled K-major shared tiles (eight warps
-//              keep enough loads in flight); warps 0-3 then run the
-//              epilogue: SiLU gate, W3 projection of this hidden block.
+//              keep enough loads in flight), then run the epilogue: SiLU
+//              gate, W3 projection of this hidden block.
 //   warp 8     allocates tensor memory and issues the MMAs (one thread).
 //   warp 9     brings the pre-split, pre-swizzled weight tiles with 1-D bulk
 //              copies.
@@ -348,18 +348,21 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
     __syncwarp();
   }
 
-  // ---- epilogue (warps 0-3 own tensor-memory lanes 32w..32w+31 = tokens)
-  if (warp < 4) {
+  // ---- epilogue: producer warp w reads tensor-memory lanes 32 (w % 4).. (its
+  // 32 tokens; a warp may only read its quarter of the lanes) and half w / 4
+  // of the hidden block's columns; the halves' partial scores meet in shared
+  // memory (the stages are free: every MMA has completed)
+  if (warp < kTcProdWarps) {
+    const int q4 = warp & 3, half = warp >> 2;
     const bool ok = mbar_wait(done, 0);
     if (!ok) fail();
     tc_fence_after();
+    float z0 = 0.f, z1 = 0.f, z2 = 0.f;
     // tcgen05.ld is warp-collective: the whole warp takes the same branch
-    if (__all_sync(0xffffffffu, ok && !*(volatile int*)abort_flag)) {
-      const int row = warp * 32 + lane;
-      const int64_t tok = m0 + row;
-      const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-      float z0 = 0.f, z1 = 0.f, z2 = 0.f;
-      for (int c0 = 0; c0 < HB; c0 += 32) {
+    const bool run = __all_sync(0xffffffffu, ok && !*(volatile int*)abort_flag);
+    if (run) {
+      const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+      for (int c0 = half * (HB / 2); c0 < (half + 1) * (HB / 2); c0 += 32) {
         float h1[32], h2[32];
         tmem_ld32(lane_addr + c0, h1);
         tmem_ld32(lane_addr + HB + c0, h2);
@@ -372,6 +375,20 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
           z2 = fmaf(g, __ldg(W3 + hidden * 3 + 2), z2);
         }
       }
+    }
+    const int row = q4 * 32 + lane;
+    float* zs = reinterpret_cast<float*>(stages);
+    if (half == 1) {
+      zs[3 * row + 0] = z0;
+      zs[3 * row + 1] = z1;
+      zs[3 * row + 2] = z2;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kTcProd) : "memory");  // producer warps only
+    if (half == 0 && run) {
+      const int64_t tok = m0 + row;
+      z0 += zs[3 * row + 0];
+      z1 += zs[3 * row + 1];
+      z2 += zs[3 * row + 2];
       if (tok < T) zpart[tok * nhb + hb] = make_float4(z0, z1, z2, 0.f);
     }
   }
