@@ -625,7 +625,8 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(S, args, device)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, S.lens, seed, tokens_per_step, S.router, len(S.routers))
+        cpu = cpu_baseline(w, S.lens, seed, tokens_per_step, S.router, len(S.routers),
+                           one_core=flush)
 
     if rank == 0:
         line = {
@@ -783,10 +784,22 @@ def oracle_step_estimate(w, lens, seed, route_chunks=32, pack_tokens=32768, rout
     return t_route + t_pack + t_dec, sample, O.num_threads()
 
 
-def cpu_baseline(w, lens, seed, tokens_per_step, router="moqae", maps=1):
+def cpu_baseline(w, lens, seed, tokens_per_step, router="moqae", maps=1, one_core=False):
+    """The oracle on all host cores; with one_core (the small workloads) also
+    on a single core."""
     t, sample, cores = oracle_step_estimate(w, lens, seed, router=router, maps=maps)
-    return {"value": tokens_per_step / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": sample, "projected_s_per_step": t}
+    out = {"value": tokens_per_step / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": sample, "projected_s_per_step": t}
+    if one_core:
+        from oracle import oracle as O
+        prev = O.num_threads()
+        O.set_num_threads(1)
+        try:
+            t1, _, _ = oracle_step_estimate(w, lens, seed, router=router, maps=maps)
+        finally:
+            O.set_num_threads(prev)
+        out["one_core"] = {"value": tokens_per_step / t1, "projected_s_per_step": t1}
+    return out
 
 
 def run_reference(args, rank, world):
