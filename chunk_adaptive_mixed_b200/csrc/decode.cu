@@ -102,16 +102,28 @@ __device__ __forceinline__ uint64_t pk2u(uint32_t a, uint32_t b) {
 __device__ __forceinline__ float lo2(uint64_t v) {
   float lo, hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  (void)hi;
   return lo;
 }
 __device__ __forceinline__ float hi2(uint64_t v) {
   float lo, hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  (void)lo;
   return hi;
 }
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
@@ -780,6 +792,14 @@ __device__ __forceinline__ void split_h2(float x, float y, uint32_t& hi, uint32_
   hi = h2_bits(h);
   lo = h2_bits(__floats2half2_rn(x - hf.x, y - hf.y));
 }
+// the same for a packed f32x2 pair (one packed subtract for the remainders)
+__device__ __forceinline__ void split_h2p(uint64_t xy, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(lo2(xy), hi2(xy));
+  const float2 hf = __half22float2(h);
+  hi = h2_bits(h);
+  const uint64_t r = sub2(xy, pk2(hf.x, hf.y));
+  lo = h2_bits(__floats2half2_rn(lo2(r), hi2(r)));
+}
 
 template <int D, int QPG, int E>
 __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
@@ -1006,13 +1026,18 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
       // a tile brings a scale of a higher binade, so that p * scale * 2^-A
       // stays within fp16 (p <= 2^8, scale <= 65504); both rescalings are
       // exact powers of two
+      // scales of rows past the item's end are taken as 0 (their stage bytes
+      // are stale and need not be numbers); p is 0 there as well, so those
+      // rows add exactly 0 below
       float2 vsm[NG][2];
       float smax = 0.f;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
-        vsm[g][0] = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r0 * G::SROW + 4 * g));
-        vsm[g][1] = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::VSOFF + r1 * G::SROW + 4 * g));
-        smax = fmaxf(smax, fmaxf(v0 ? vsm[g][0].x : 0.f, v1 ? vsm[g][1].x : 0.f));
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(st + G::VSOFF + r0 * G::SROW + 4 * g);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(st + G::VSOFF + r1 * G::SROW + 4 * g);
+        vsm[g][0] = half2_bits_to_float2(v0 ? b0 : 0u);
+        vsm[g][1] = half2_bits_to_float2(v1 ? b1 : 0u);
+        smax = fmaxf(smax, fmaxf(vsm[g][0].x, vsm[g][1].x));
       }
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
@@ -1028,18 +1053,20 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
         abits = eb;
       }
       const float down = __uint_as_float(0x7F000000u - abits);  // 2^-A
+      // (head slot 2 tig, 2 tig + 1) pairs of p for rows r0 and r1, and p * 2^-A
+      const uint64_t pp0 = pk2(p[0], p[1]), pp1 = pk2(p[2], p[3]);
+      const uint64_t pd0 = mul2(pp0, pk2(down, down)), pd1 = mul2(pp1, pk2(down, down));
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         const float2 sm0 = vsm[g][0], sm1 = vsm[g][1];
-        // rows past the item's end contribute exactly 0, never 0 * stale bytes
-        const float s0 = sm0.x * down, s1 = sm1.x * down;
-        const float x0 = v0 ? p[0] * s0 : 0.f, x1 = v0 ? p[1] * s0 : 0.f;
-        const float x2 = v1 ? p[2] * s1 : 0.f, x3 = v1 ? p[3] * s1 : 0.f;
-        vb[g][0] += (v0 ? p[0] * sm0.y : 0.f) + (v1 ? p[2] * sm1.y : 0.f);
-        vb[g][1] += (v0 ? p[1] * sm0.y : 0.f) + (v1 ? p[3] * sm1.y : 0.f);
+        const uint64_t xa = mul2(pd0, pk2(sm0.x, sm0.x));  // (x0, x1): row r0
+        const uint64_t xb = mul2(pd1, pk2(sm1.x, sm1.x));  // (x2, x3): row r1
+        const uint64_t vbg = fma2(pp1, pk2(sm1.y, sm1.y), fma2(pp0, pk2(sm0.y, sm0.y), pk2(vb[g][0], vb[g][1])));
+        vb[g][0] = lo2(vbg);
+        vb[g][1] = hi2(vbg);
         uint32_t hi0, lo0, hi1, lo1;
-        split_h2(x0, x1, hi0, lo0);
-        split_h2(x2, x3, hi1, lo1);
+        split_h2p(xa, hi0, lo0);
+        split_h2p(xb, hi1, lo1);
         const uint32_t bh0 = movm_t(hi0), bh1 = movm_t(hi1), bl0 = movm_t(lo0), bl1 = movm_t(lo1);
 #pragma unroll
         for (int mm = 0; mm < 2; ++mm) {
@@ -1091,10 +1118,10 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
       vb[g][1] += __shfl_xor_sync(0xffffffffu, vb[g][1], off);
     }
   }
-#pragma unroll
   // 2^A (and 2^24 for INT4 codes entered as c * 2^-24)
   const float up = (E == 0 || abits == 0u) ? 1.f
                    : __uint_as_float(abits) * (E == 1 ? 16777216.0f : 1.0f);
+#pragma unroll
   for (int hj = 0; hj < 2; ++hj) {
     const int h = 2 * tig + hj;
     if (h < QPG) {
