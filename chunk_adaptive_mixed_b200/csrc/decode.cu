@@ -100,15 +100,15 @@ __device__ __forceinline__ uint64_t pk2u(uint32_t a, uint32_t b) {
   return d;
 }
 __device__ __forceinline__ float lo2(uint64_t v) {
-  float lo, hi;
+  float lo;
+  [[maybe_unused]] float hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  (void)hi;
   return lo;
 }
 __device__ __forceinline__ float hi2(uint64_t v) {
-  float lo, hi;
+  [[maybe_unused]] float lo;
+  float hi;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  (void)lo;
   return hi;
 }
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
@@ -854,7 +854,9 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
 
   // ---- query operand (B of the score MMA): head slot gid, zero past QPG
   uint32_t qb[NK][2];
-  float qsum[NG][2];
+  // per group, the (head slot 2 tig, 2 tig + 1) pair of query sums; for INT4
+  // in units of 2^24 (the codes enter as c * 2^-24, see score_scale)
+  uint64_t qsum2[NG];
   {
     const bool hv = gid < QPG;
     const __half* qh = q + qbase + (int64_t)(hv ? gid : 0) * D;
@@ -886,11 +888,13 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
       part[g] += __shfl_xor_sync(0xffffffffu, part[g], 1);
       part[g] += __shfl_xor_sync(0xffffffffu, part[g], 2);
       // sums of heads 2 tig and 2 tig + 1 live in lanes 8 tig and 8 tig + 4
-      qsum[g][0] = __shfl_sync(0xffffffffu, part[g], 8 * tig);
-      qsum[g][1] = __shfl_sync(0xffffffffu, part[g], 8 * tig + 4);
+      const float u = E == 1 ? 1.0f / 16777216.0f : 1.0f;
+      qsum2[g] = pk2(__shfl_sync(0xffffffffu, part[g], 8 * tig) * u,
+                     __shfl_sync(0xffffffffu, part[g], 8 * tig + 4) * u);
     }
   }
 
+  const float score_scale = scale_log2 * (E == 1 ? 16777216.0f : 1.0f);
   float o[NK][4];
   float vb[NG][2];
   float mrun[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
@@ -913,8 +917,11 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
     const bool v0 = r0 < nv, v1 = r1 < nv;
 
     // ---- scores: C rows = tokens (r0, r1), columns = head slots (2 tig, 2 tig + 1)
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    // scores of rows (r0, r1) x head slots (2 tig, 2 tig + 1), as f32x2 pairs;
+    // INT4 scores in units of 2^-24
+    uint64_t s01, s23;
     if constexpr (E == 0) {
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t kbase = smem_addr(st + G::KOFF);
       const int j = lane >> 3;
       const uint32_t arow = kbase + ((lane & 7) + (j & 1) * 8) * G::KROW + (j >> 1) * 16;
@@ -924,7 +931,25 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
         ldsm_x4(a, arow + kk * 32);
         mma16816(s4, a[0], a[1], a[2], a[3], qb[kk][0], qb[kk][1]);
       }
+      s01 = pk2(s4[0], s4[1]);
+      s23 = pk2(s4[2], s4[3]);
     } else {
+      // the rows' (scale, min) pairs of all groups, one vector load per row
+      uint32_t ks0[NG], ks1[NG];
+      if constexpr (NG == 4) {
+        const uint4 a = *reinterpret_cast<const uint4*>(st + G::KSOFF + r0 * G::SROW);
+        const uint4 b = *reinterpret_cast<const uint4*>(st + G::KSOFF + r1 * G::SROW);
+        ks0[0] = a.x; ks0[1] = a.y; ks0[2] = a.z; ks0[3] = a.w;
+        ks1[0] = b.x; ks1[1] = b.y; ks1[2] = b.z; ks1[3] = b.w;
+      } else {
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          ks0[g] = *reinterpret_cast<const uint32_t*>(st + G::KSOFF + r0 * G::SROW + 4 * g);
+          ks1[g] = *reinterpret_cast<const uint32_t*>(st + G::KSOFF + r1 * G::SROW + 4 * g);
+        }
+      }
+      s01 = 0ull;
+      s23 = 0ull;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -946,26 +971,19 @@ __device__ __forceinline__ void mma_item(const unsigned char* __restrict__ regk,
             mma16816(acc, a0, a1, a2, a3, qb[2 * g + hh][0], qb[2 * g + hh][1]);
           }
         }
-        float2 sm0 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r0 * G::SROW + 4 * g));
-        float2 sm1 = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(st + G::KSOFF + r1 * G::SROW + 4 * g));
-        if constexpr (E == 1) {  // codes entered as c * 2^-24
-          sm0.x *= 16777216.0f;
-          sm1.x *= 16777216.0f;
-        }
-        s4[0] = fmaf(sm0.x, acc[0], fmaf(sm0.y, qsum[g][0], s4[0]));
-        s4[1] = fmaf(sm0.x, acc[1], fmaf(sm0.y, qsum[g][1], s4[1]));
-        s4[2] = fmaf(sm1.x, acc[2], fmaf(sm1.y, qsum[g][0], s4[2]));
-        s4[3] = fmaf(sm1.x, acc[3], fmaf(sm1.y, qsum[g][1], s4[3]));
+        const float2 sm0 = half2_bits_to_float2(ks0[g]), sm1 = half2_bits_to_float2(ks1[g]);
+        s01 = fma2(pk2(acc[0], acc[1]), pk2(sm0.x, sm0.x), fma2(qsum2[g], pk2(sm0.y, sm0.y), s01));
+        s23 = fma2(pk2(acc[2], acc[3]), pk2(sm1.x, sm1.x), fma2(qsum2[g], pk2(sm1.y, sm1.y), s23));
       }
     }
 
     // ---- online softmax per head slot (log2 domain, lazily moved reference;
     // rows past the item's end hold stale bytes and are masked, never used)
     float sc[4];
-    sc[0] = v0 ? s4[0] * scale_log2 : -INFINITY;
-    sc[1] = v0 ? s4[1] * scale_log2 : -INFINITY;
-    sc[2] = v1 ? s4[2] * scale_log2 : -INFINITY;
-    sc[3] = v1 ? s4[3] * scale_log2 : -INFINITY;
+    sc[0] = v0 ? lo2(s01) * score_scale : -INFINITY;
+    sc[1] = v0 ? hi2(s01) * score_scale : -INFINITY;
+    sc[2] = v1 ? lo2(s23) * score_scale : -INFINITY;
+    sc[3] = v1 ? hi2(s23) * score_scale : -INFINITY;
     float tm[2] = {fmaxf(sc[0], sc[2]), fmaxf(sc[1], sc[3])};
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
