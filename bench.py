@@ -82,8 +82,8 @@ def measured_peaks():
 # profiles/), valid only for the pack kernel source (pack.cu) with this
 # SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "a3a08a04cf53dd5d42e1fb6231e64fe083732404b654f9da30ac00c4e060144c",
-                "bytes_per_launch": 2148122624 + 843587328}
+                "sha256": "c253ef3387d2e12705941d3c52a9e0f19e3d2e8e6e0064e3a1df03f3c412361d",
+                "bytes_per_launch": 2148355840 + 843005952}
 
 
 def pack_sources_sha256():
