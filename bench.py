@@ -82,7 +82,7 @@ def measured_peaks():
 # profiles/), valid only for the pack kernel source (pack.cu) with this
 # SHA-256.
 PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "c253ef3387d2e12705941d3c52a9e0f19e3d2e8e6e0064e3a1df03f3c412361d",
+                "sha256": "8a9960beeb72542fc97eda5327348a6f19cbddb77bc9d45c775727e1d8600141",
                 "bytes_per_launch": 2148355840 + 843005952}
 
 
