@@ -577,7 +577,7 @@ decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
   for (int i = 0; i < PER_LANE; ++i) acc[i] = 0.f;
   // kU items per round, all loaded before any is merged (independent loads
   // in flight instead of one dependent load at a time)
-  constexpr int kU = 4;
+  constexpr int kU = 8;
   for (int it0 = i0 + warp; it0 < i1; it0 += NW * kU) {
     float2 ml[kU];
     float v[kU][PER_LANE];
