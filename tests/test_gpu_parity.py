@@ -30,6 +30,10 @@ CASES = {
     "gqa2_f16": Case(np.array([700, 64, 1, 0], np.int32), 4, 2, 128, 64, "f16"),
     "gqa8_d128": Case(np.array([2000, 33], np.int32), 16, 2, 128, 128, "f16"),
     "gqa4_d64": Case(np.array([1500, 17, 96], np.int32), 8, 2, 64, 32, "f16"),
+    # fp32 queries with 4 and 8 query heads per kv-head: the CUDA-core kernel
+    # with 8- and 4-dim lane slices (code words of 1 to 4 bytes)
+    "gqa4_f32_d64": Case(np.array([900, 31, 64], np.int32), 8, 2, 64, 32, "f32"),
+    "gqa8_f32_d128": Case(np.array([700, 129], np.int32), 16, 2, 128, 64, "f32"),
 }
 
 MAPS = {"mixed": (0.2, 0.5, 0.3), "fp16": (1, 0, 0), "int4": (0, 1, 0), "int2": (0, 0, 1)}
@@ -43,7 +47,8 @@ def _map(case, mix, seed=0):
 @pytest.mark.parametrize("mapname", list(MAPS))
 def test_layout_pack_decode_parity(name, mapname):
     case = CASES[name]
-    if mapname != "mixed" and name not in ("ragged_gqa4", "tiny_like_f32", "gqa8_d128", "gqa4_d64"):
+    if mapname != "mixed" and name not in ("ragged_gqa4", "tiny_like_f32", "gqa8_d128", "gqa4_d64",
+                                           "gqa4_f32_d64", "gqa8_f32_d128"):
         pytest.skip("single-precision maps run on two cases")
     cmap = _map(case, MAPS[mapname], seed=zlib.crc32(name.encode()) & 0xFFFF)
     K, V, q = random_kv(case, seed=len(name))
