@@ -441,6 +441,51 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
       av[h][2 * j + 1] =
           hi2(acc[h][j]) * (E == 0 ? 1.f : pow2f(149 - kWExp - code_off<BITS>(2 * j + 1)));
     }
+  if constexpr (QPG == 1) {
+    // One query head: merge through the warp's ring, idle now (every copy has
+    // landed and been read).  Each lane stores its slice (SL dims) with its
+    // token lane's (m, l, bias); then lane i combines dims DPL i.. over the
+    // TPW token lanes of their slice.
+    constexpr int ROW = SL + 4;  // floats per lane: av[SL], m, l, bias, pad
+    constexpr int DPL = D / 32;  // output dims per lane
+    float* smf = reinterpret_cast<float*>(ring);
+    float* row = smf + lane * ROW;
+#pragma unroll
+    for (int j = 0; j < SL; j += 4)
+      *reinterpret_cast<float4*>(row + j) = make_float4(av[0][j], av[0][j + 1], av[0][j + 2], av[0][j + 3]);
+    *reinterpret_cast<float4*>(row + SL) = make_float4(m[0], l[0], bias[0], 0.f);
+    __syncwarp();
+    const int d0 = lane * DPL;
+    const int sld = d0 / SL, o = d0 % SL;
+    float M = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < TPW; ++t) M = fmaxf(M, smf[(t * LPT + sld) * ROW + SL]);
+    float L = 0.f, Bs = 0.f, ad[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) ad[i] = 0.f;
+#pragma unroll
+    for (int t = 0; t < TPW; ++t) {
+      const float* src = smf + (t * LPT + sld) * ROW;
+      const float4 mlb = *reinterpret_cast<const float4*>(src + SL);
+      const float a = mlb.x == -INFINITY ? 0.f : ex2_ftz(mlb.x - M);
+      L = fmaf(a, mlb.y, L);
+      Bs = fmaf(a, mlb.z, Bs);
+      if constexpr (DPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src + o);
+        ad[0] = fmaf(a, v.x, ad[0]);
+        ad[1] = fmaf(a, v.y, ad[1]);
+        ad[2] = fmaf(a, v.z, ad[2]);
+        ad[3] = fmaf(a, v.w, ad[3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) ad[i] = fmaf(a, src[o + i], ad[i]);
+      }
+    }
+    float* dst = ws_acc + (size_t)w * D + d0;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) dst[i] = ad[i] + Bs;
+    if (lane == 0) ws_ml[w] = make_float2(M, L);
+  } else {
 #pragma unroll
   for (int off = LPT; off < 32; off <<= 1) {
 #pragma unroll
@@ -476,7 +521,8 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
 #pragma unroll
     for (int h = 0; h < QPG; ++h) ws_ml[(size_t)w * QPG + h] = make_float2(m[h], l[h]);
   }
-  __syncwarp();
+  }
+  __syncwarp();  // (one query head: the ring is read before the next item's copies refill it)
 }
 
 __device__ __forceinline__ int find_item_seq(const unsigned char* layout, int B, int64_t bs) {
