@@ -141,6 +141,13 @@ cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layo
                           const void* packed, const void* q, int q_dtype, float softmax_scale,
                           float* out, void* workspace, size_t workspace_bytes,
                           unsigned int* status, cudaStream_t stream, bool partial = false);
+// Per-item partial results of decode on the tensor cores (one query head per
+// kv-head, fp16 queries, head_dim 128): the same workspace records as the
+// CUDA-core kernel; the counter is zeroed on the stream first.
+cudaError_t launch_decode_mha(int64_t capacity_items, const unsigned char* layout,
+                              const unsigned char* packed, const __half* q, float scale_log2,
+                              float* ws_acc, float2* ws_ml, unsigned int* counter,
+                              unsigned int* status, cudaStream_t stream);
 cudaError_t launch_combine_partials(int P, int B, int Hq, int D, const float* parts, float* out,
                                     cudaStream_t stream);
 

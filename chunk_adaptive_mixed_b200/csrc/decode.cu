@@ -31,7 +31,7 @@
 //          acc[d]) of every head goes to the workspace.
 // decode_combine_kernel — one warp per (b, query head) merges the partials of
 // all items of (b, g) with the usual max-rescaling.
-#include "common.cuh"
+#include "decode_ptx.cuh"
 
 namespace mqkv {
 namespace {
@@ -69,74 +69,6 @@ constexpr int stage_bytes() {
 template <int D, int QPG>
 constexpr size_t decode_smem_bytes() {
   return (size_t)kDecWarps * kRing * stage_bytes<D, QPG>();
-}
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t bits) {
-  __half2 h;
-  *reinterpret_cast<uint32_t*>(&h) = bits;
-  return __half22float2(h);
-}
-
-// ---- packed fp32 pairs (sm_100 f32x2 arithmetic, round to nearest)
-// Pairs are built and taken apart with register-pair moves (no shifts or ORs).
-__device__ __forceinline__ uint64_t pk2(float a, float b) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a), "f"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t pk2u(uint32_t a, uint32_t b) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ float lo2(uint64_t v) {
-  float lo;
-  [[maybe_unused]] float hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float hi2(uint64_t v) {
-  [[maybe_unused]] float lo;
-  float hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-// 2^x by the hardware approximation (max error 2 ulp), results below 2^-126
-// flushed to zero: softmax weights that small do not register in the sums.
-__device__ __forceinline__ float ex2_ftz(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
 }
 
 // Code extraction by masking in place.  A 32-bit pattern below 2^24, read as
@@ -525,16 +457,6 @@ __device__ __forceinline__ void run_item(const unsigned char* __restrict__ regk,
   __syncwarp();  // (one query head: the ring is read before the next item's copies refill it)
 }
 
-__device__ __forceinline__ int find_item_seq(const unsigned char* layout, int B, int64_t bs) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) / 2;
-    const mq_seq_layout* r =
-        reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(mid));
-    if (r->item_begin[0] <= bs) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
 
 // Each warp is an independent worker: it takes the next work item from a
 // counter in the workspace whenever it finishes one, and streams each item
@@ -780,33 +702,6 @@ template <int D>
 constexpr size_t mma_smem_bytes() {
   return (size_t)kMmaWarps * kMmaRing;
 }
-
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
 // byte j of w as [b, 0x64, b, 0x64]: two fp16 values 1024 + (low bits of b)
 __device__ __forceinline__ uint32_t spread2(uint32_t w, int j) {
@@ -1289,7 +1184,10 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
     }
     return cudaSuccess;
   };
-  if constexpr (kMma)
+  if constexpr (D == 128 && QPG == 1 && QDT == MQ_F16)
+    err = launch_decode_mha(cap, layout, packed, static_cast<const __half*>(q), scale_log2, ws_acc,
+                            ws_ml, counter, status, stream);
+  else if constexpr (kMma)
     err = run(decode_mma_kernel<D, QPG>, static_cast<const __half*>(q));
   else
     err = run(decode_partial_kernel<D, QPG, QDT>, q);

@@ -28,7 +28,11 @@ std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once
-// per device (the first call on each device does the lookup).
+// per device (the first call on each device does the lookup).  The cached
+// address belongs to the device's current primary context: after
+// cudaDeviceReset the module is loaded afresh and the cache is stale, so a
+// process that resets a device must not call mq_decode_attn_noalloc again on
+// it.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -70,6 +74,9 @@ extern "C" mq_status mq_decode_attn_noalloc(const mq_shape* shape, const int32_t
                                 "mq_decode_attn_noalloc: address of the scratch array: %s",
                                 cudaGetErrorString(err));
   }
+  // With no scratch (need == 0: invalid arguments) the capacity passed is 0,
+  // so mq_decode_attn's argument checks report exactly what they report for a
+  // caller with no workspace.
   return mq_decode_attn(shape, h_seq_lens, layout, packed, q, q_dtype, softmax_scale, out,
-                        scratch, (size_t)MQ_NOALLOC_SCRATCH_BYTES, stream);
+                        scratch, scratch ? (size_t)MQ_NOALLOC_SCRATCH_BYTES : 0, stream);
 }

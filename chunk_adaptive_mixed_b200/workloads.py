@@ -17,7 +17,8 @@ datasets exist here: every tensor is random, of that model's shape):
                     shape and distribution as llama2_7b_layer, K/V of layer l
                     drawn from seed + l
   llama2_13b_128k   40 layers, 1 x 131072 tokens, 40 heads x 128, chunk 256,
-                    D=5120, H=256, fp16; ~5/35/60
+                    D=5120, H=256, fp16; ~5/35/60; K/V drawn and packed one
+                    layer at a time, only the packed cache resident
   llama3_8b_gqa     1 layer, 64 sequences of lengths uniform in [2048, 16384],
                     32 query / 8 KV heads x 128, chunk 128, D=4096, H=256, fp16;
                     ~15/60/25; a fresh fp16 query per decode step, 100 steps
@@ -72,6 +73,9 @@ class Workload:
     sink_scale: float                  # token 0's key is multiplied by this
     decode_steps: int = 1
     chunk_corr: float = 0.9
+    # K/V drawn and packed one layer at a time (only the packed cache of every
+    # layer stays resident), instead of every layer's K/V resident at once
+    kv_streamed: bool = False
 
     @property
     def torch_dtype(self):
@@ -106,7 +110,8 @@ WORKLOADS = {
         head_dim=128, chunk_len=256, router_dim=5120, router_hidden=256, kv_dtype="f16",
         seq_len=131072, seq_len_range=None, target_mix=(0.05, 0.35, 0.60),
         router_bias=(0.0, 0.88, 0.94),
-        outlier_channels=None, num_outlier_channels=4, outlier_scale=10.0, sink_scale=5.0),
+        outlier_channels=None, num_outlier_channels=4, outlier_scale=10.0, sink_scale=5.0,
+        kv_streamed=True),
     "llama3_8b_gqa": Workload(
         name="llama3_8b_gqa", layers=1, num_seqs=64, num_q_heads=32, num_kv_heads=8,
         head_dim=128, chunk_len=128, router_dim=4096, router_hidden=256, kv_dtype="f16",

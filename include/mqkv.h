@@ -381,7 +381,9 @@ mq_status mq_decode_attn(const mq_shape* shape, const int32_t* h_seq_lens,
  *          MQ_NOALLOC_SCRATCH_BYTES; otherwise errors as mq_decode_attn.
  *   Set-up: the first call on each device looks up the array's device
  *          address (cudaGetSymbolAddress) with that device current; make that
- *          first call before any stream capture begins.
+ *          first call before any stream capture begins.  The address is kept
+ *          for the life of the process: after cudaDeviceReset on a device,
+ *          do not call this function on that device again.
  *   Sharing: every call uses the same array, which keeps what the last call
  *          wrote.  Calls whose work overlaps on the GPU (other streams, other
  *          host threads) race on it and corrupt each other's results.

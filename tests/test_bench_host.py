@@ -1,0 +1,61 @@
+"""Host-side logic of the benchmark that needs no GPU: the routing sample, the
+workload description both arms print, and the reference arm's line."""
+import json
+import subprocess
+import sys
+import os
+
+import numpy as np
+
+import bench
+from chunk_adaptive_mixed_b200 import workloads as W
+
+
+def test_route_sample_spreads_over_the_batch():
+    for N, count in ((512, 128), (4608, 128), (16, 128), (1, 8), (1024, 8)):
+        c = bench.route_sample_chunks(N, count)
+        assert c == sorted(set(c))
+        assert all(0 <= x < N for x in c)
+        assert len(c) <= max(min(count, N), 1)
+        assert 0 in c and N - 1 in c
+        if N >= 4 * count:
+            # groups cover the whole batch: no half of it is left out
+            assert min(c) < N // 4 and max(c) >= 3 * N // 4
+
+
+def test_both_arms_print_the_same_config():
+    w = W.get("llama2_13b_128k")
+    lens = W.seq_lens(w, 0)
+    a = bench.line_config(w, lens, True, "moqae", 0.0, False, False, 1)
+    b = bench.line_config(w, lens, True, "moqae", 0.0, False, False, 1)
+    assert a == b
+    assert a["workload"] == "llama2_13b_128k" and a["layers"] == 40
+    assert "only the packed cache" in a["kv"]
+    assert "sum of the library spans" in a["step_time"]
+    small = bench.line_config(W.get("llama2_7b_layer"), W.seq_lens(W.get("llama2_7b_layer"), 0),
+                              True, "moqae", 0.0, False, False, 1)
+    assert small["l2"].startswith("2 x L2 buffer")
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    assert bench.DEFAULT_WORKLOAD == "llama2_13b_128k"
+    assert W.get(bench.DEFAULT_WORKLOAD).kv_streamed
+
+
+def test_reference_arm_line_on_a_small_workload():
+    # the oracle on a bounded sample: ms_per_step is the sample's measured
+    # time, the value its projection to the full step, the config the same
+    # dict our arm prints
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], cwd=root, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s"
+    w = W.get("tiny")
+    assert line["config"] == json.loads(json.dumps(
+        bench.line_config(w, W.seq_lens(w, 0), True, "moqae", 0.0, False, False, 1)))
+    assert line["ms_per_step"] <= line["projected_ms_per_full_step"] + 1e-9
+    assert line["sample_wall_s"] * 1e3 >= line["ms_per_step"] * line["steps"] * 0.99
+    assert np.isfinite(line["value"]) and line["value"] > 0

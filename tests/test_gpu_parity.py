@@ -34,6 +34,10 @@ CASES = {
     # with 8- and 4-dim lane slices (code words of 1 to 4 bytes)
     "gqa4_f32_d64": Case(np.array([900, 31, 64], np.int32), 8, 2, 64, 32, "f32"),
     "gqa8_f32_d128": Case(np.array([700, 129], np.int32), 16, 2, 128, 64, "f32"),
+    # one query head per kv-head, fp16 queries, d = 128: the tensor-core
+    # kernel of that case (16-token stages: tails of 1, 15, 16, 17 tokens)
+    "mha_f16_d128": Case(np.array([0, 1, 15, 16, 17, 127, 129, 1000, 3000], np.int32), 4, 4, 128,
+                         32, "f16"),
 }
 
 MAPS = {"mixed": (0.2, 0.5, 0.3), "fp16": (1, 0, 0), "int4": (0, 1, 0), "int2": (0, 0, 1)}
@@ -48,7 +52,7 @@ def _map(case, mix, seed=0):
 def test_layout_pack_decode_parity(name, mapname):
     case = CASES[name]
     if mapname != "mixed" and name not in ("ragged_gqa4", "tiny_like_f32", "gqa8_d128", "gqa4_d64",
-                                           "gqa4_f32_d64", "gqa8_f32_d128"):
+                                           "gqa4_f32_d64", "gqa8_f32_d128", "mha_f16_d128"):
         pytest.skip("single-precision maps run on two cases")
     cmap = _map(case, MAPS[mapname], seed=zlib.crc32(name.encode()) & 0xFFFF)
     K, V, q = random_kv(case, seed=len(name))
@@ -126,7 +130,10 @@ def test_route_without_bias_and_zero_w1():
 @pytest.mark.parametrize("name", ["tiny", "llama2_7b_layer"])
 def test_end_to_end_small_workloads(name):
     """route -> layout -> pack -> decode on the workload's own inputs, GPU vs
-    oracle, each side with its own routing map."""
+    oracle.  Routing is compared as in the router tests; layout, pack and
+    decode then run on the oracle's map on both sides, which equals the GPU's
+    own map unless a near-tie chunk flipped, so no branch ends without a
+    pack and decode comparison."""
     w = W.get(name)
     lens = W.seq_lens(w)
     case = Case(lens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.chunk_len, w.kv_dtype)
@@ -140,18 +147,18 @@ def test_end_to_end_small_workloads(name):
                                    W3.numpy(), b3.numpy())
     near, exempt = check_route(lens, w.chunk_len, te, ce, logits, z32, z64)
     assert ce[0] == 0
-    layout = gpu_layout(case, ce)
-    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
-    out = gpu_decode(case, layout, packed, q.to(dev()))
+    print(f"{name}: {case.T} tokens routed, {near} near-tie tokens, {exempt} exempt chunks")
+    if not np.array_equal(ce, ce_o):
+        assert exempt > 0
+    # layout, pack and decode run on the oracle's map: the GPU's own map
+    # unless a near-tie chunk flipped (the oracle never receives the GPU's map)
     ref = O.pack(case.Hkv, case.d, case.L, lens, ce_o, K.numpy(), V.numpy())
     want = O.decode(case.Hq, case.Hkv, case.d, case.L, lens, ce_o, ref, q.numpy())
-    if np.array_equal(ce, ce_o):
-        assert np.array_equal(packed[:pb].cpu().numpy(), ref)
-        check_attention(out, want, name)
-    else:
-        # a near-tie chunk flipped: the two sides quantised that chunk
-        # differently, so only the routing check above applies
-        assert exempt > 0
+    layout = gpu_layout(case, ce_o)
+    check_layout(case, layout.cpu().numpy(), ce_o)
+    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+    assert np.array_equal(packed[:pb].cpu().numpy(), ref)
+    check_attention(gpu_decode(case, layout, packed, q.to(dev())), want, name)
 
 
 def test_device_checks_without_faults():
@@ -207,20 +214,22 @@ def test_routing_sharing_off_gives_each_layer_its_own_map_and_layout():
                                    b3.to(dev()))
         ce_o, _, z32, z64 = O.route(lens, case.L, C.numpy(), W1.numpy(), W2.numpy(), W3.numpy(),
                                     b3.numpy())
-        _, exempt = check_route(lens, case.L, te, ce, logits, z32, z64)
+        near, exempt = check_route(lens, case.L, te, ce, logits, z32, z64)
+        print(f"layer {layer}: {near} near-tie tokens, {exempt} exempt chunks")
+        if not np.array_equal(ce, ce_o):
+            assert exempt > 0
         maps.append(ce_o)
         K, V, q = random_kv(case, seed=100 + layer)
-        layout = gpu_layout(case, ce)                      # the GPU's own map
+        # layout, pack and decode on the oracle's map (identical to the GPU's
+        # unless a near-tie chunk flipped); the oracle side uses its own map
+        layout = gpu_layout(case, ce_o)
         packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
         out = gpu_decode(case, layout, packed, q.to(dev()))
         ref = O.pack(case.Hkv, case.d, case.L, lens, ce_o, K.numpy(), V.numpy())
         want = O.decode(case.Hq, case.Hkv, case.d, case.L, lens, ce_o, ref, q.numpy())
-        if np.array_equal(ce, ce_o):
-            check_layout(case, layout.cpu().numpy(), ce_o)
-            assert np.array_equal(packed[:pb].cpu().numpy(), ref)
-            check_attention(out, want, f"layer {layer}")
-        else:
-            assert exempt > 0
+        check_layout(case, layout.cpu().numpy(), ce_o)
+        assert np.array_equal(packed[:pb].cpu().numpy(), ref)
+        check_attention(out, want, f"layer {layer}")
     assert any(not np.array_equal(maps[0], m) for m in maps[1:])
 
 
@@ -339,9 +348,10 @@ def test_decode_with_very_large_groups(hq, hkv):
     check_attention(out / scale, want / scale, "large groups (relative to the output range)")
 
 
-def test_decode_with_tiny_values():
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (4, 4)])
+def test_decode_with_tiny_values(hq, hkv):
     # every group tiny (scales ~1e-6): the tensor-core path keeps its relative accuracy
-    case = Case(np.array([700, 90], np.int32), 8, 2, 128, 64, "f16")
+    case = Case(np.array([700, 90], np.int32), hq, hkv, 128, 64, "f16")
     K, V, q = random_kv(case, seed=91)
     V = (V.float() * 2e-5).half()
     cmap = _map(case, MAPS["mixed"], seed=6)
@@ -352,3 +362,26 @@ def test_decode_with_tiny_values():
     want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
     scale = np.abs(want).max()
     check_attention(out / scale, want / scale, "tiny values (relative to the output range)")
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2)])
+def test_decode_query_extremes(hq, hkv):
+    # queries at the edges of fp16: all zero, a huge element beside tiny and
+    # subnormal ones, every element subnormal; the tensor-core kernels scale
+    # each query by a power of two before it enters an fp16 operand
+    case = Case(np.array([600, 77, 33], np.int32), hq, hkv, 128, 64, "f16")
+    K, V, q = random_kv(case, seed=123)
+    qf = q.float()
+    qf[0, 0] = 0.0
+    qf[1, 0] = torch.where(torch.arange(case.d) % 3 == 0, 3e-7, 1e-3)
+    qf[1, 0, 5] = 30000.0
+    qf[2, 0] = torch.linspace(-1.0, 1.0, case.d) * 2.0 ** -15
+    q = qf.half()
+    K = (K.float() * 0.01).half()      # keeps the 30000 query's scores finite and spread
+    cmap = _map(case, MAPS["mixed"], seed=8)
+    layout = gpu_layout(case, cmap)
+    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+    ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, K.numpy(), V.numpy())
+    out = gpu_decode(case, layout, packed, q.to(dev()))
+    want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
+    check_attention(out, want, "query extremes")
