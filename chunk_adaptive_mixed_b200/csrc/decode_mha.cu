@@ -30,81 +30,52 @@
 // with o its bit offset there; codes at offsets that would reach 2^11 are
 // first shifted down (INT4 by 8, INT2 by 10).  The power of two 2^o of each
 // operand slot is divided out of the matching query element (scores; the
-// query is first brought to [2^14, 2^15) by one power of two per item so the
-// divided elements stay normal) or out of the finished accumulator (values).
-// For the value product the A operand pairs two tokens of one dim: byte
-// permutes interleave the 16-bit halves of two token rows, then masks pick
-// each dim's code pair.
+// query is first brought to [2^14, 2^15) by one power of two so the divided
+// elements stay normal) or out of the finished accumulator (values).  For the
+// value product the A operand pairs two tokens of one dim: byte permutes
+// interleave the 16-bit halves of two token rows, then masks pick each dim's
+// code pair.
 //
-// One warp per CTA (12 per SM) is an independent persistent worker: it takes
-// work items from an atomic counter and streams each item through its own
-// cp.async ring of 16-token stages.  The stage layout keeps every lane's
-// shared-memory reads conflict-free without padding for the quantised tiles
-// (FP16 rows are padded for ldmatrix).
+// Work: one warp per CTA (12 per SM) is a persistent worker.  Work items are
+// numbered region by region — (sequence, segment, kv-head), then the items of
+// that region in token order — and a worker claims a group of consecutive
+// items from an atomic counter, the group shrinking as the work runs out
+// (guided self-scheduling: long streams early, a short tail).  Consecutive
+// items of one region form one run: the worker streams the run's token range
+// through its cp.async ring (32-token stages for INT4 / INT2, 16-token stages
+// for FP16) without draining the ring at item boundaries, and writes each
+// item's partial record when the item's last stage is done.  Every item is
+// computed from a fresh state, so its record does not depend on which worker
+// took it or on the grouping.  Quantised stages are laid out so that every
+// lane's shared-memory reads are conflict-free without padding; FP16 rows are
+// padded for ldmatrix.
 #include "decode_ptx.cuh"
 
 namespace mqkv {
 namespace {
 
-constexpr int kTcTile = 16;        // tokens per stage
-constexpr int kTcRing = 17408;     // shared bytes per worker warp
-constexpr int kTcCtasPerSm = 12;   // one-warp CTAs resident per SM
-constexpr float kTcRescale = 8.0f; // lazy softmax reference: weights stay below 2^8
+constexpr int kTcRing = 17408;      // shared bytes per worker warp
+constexpr int kTcCtasPerSm = 12;    // one-warp CTAs resident per SM
+constexpr float kTcRescale = 8.0f;  // lazy softmax reference: weights stay below 2^8
+constexpr int kTcMaxGroup = 8;      // items per claim at most
 
 template <int E>
 struct TG {  // stage geometry at head_dim 128
   static constexpr int BITS = E == 0 ? 16 : (E == 1 ? 4 : 2);
+  static constexpr int SUB = E == 0 ? 1 : 2;             // 16-token subtiles per stage
+  static constexpr int TOK = 16 * SUB;                   // tokens per stage
   static constexpr int CROW = 128 * BITS / 8;            // code bytes of a token row
   static constexpr int KROW = E == 0 ? CROW + 16 : CROW; // staged pitch
   static constexpr int SROW = E == 0 ? 0 : 16;           // (scale, min) bytes of a row
   static constexpr int KOFF = 0;
-  static constexpr int VOFF = kTcTile * KROW;
-  static constexpr int KSOFF = 2 * kTcTile * KROW;
-  static constexpr int VSOFF = KSOFF + kTcTile * SROW;
-  static constexpr int STAGE = VSOFF + kTcTile * SROW;
+  static constexpr int VOFF = TOK * KROW;
+  static constexpr int KSOFF = 2 * TOK * KROW;
+  static constexpr int VSOFF = KSOFF + TOK * SROW;
+  static constexpr int STAGE = VSOFF + TOK * SROW;
   static constexpr int STAGES = kTcRing / STAGE < 8 ? kTcRing / STAGE : 8;
   static constexpr int CU = CROW / 16;                   // 16-byte units per code row
 };
-static_assert(TG<0>::STAGES >= 2 && TG<1>::STAGES >= 4 && TG<2>::STAGES >= 4, "ring too small");
-
-// Copies of one stage (rows [row0, row0 + nv) of the item's regions) into st.
-template <int E>
-__device__ __forceinline__ void tc_issue(unsigned char* st, const unsigned char* regk,
-                                         const unsigned char* regv, uint64_t soff, int64_t row0,
-                                         int nv, int lane) {
-  using G = TG<E>;
-  if constexpr (E == 0) {
-    // 16 units per row; lane covers rows r, r + 2, ... at column c
-    const int r = lane >> 4, c = (lane & 15) * 16;
-    const unsigned char* sk = regk + (row0 + r) * G::CROW + c;
-    const unsigned char* sv = regv + (row0 + r) * G::CROW + c;
-    unsigned char* dk = st + G::KOFF + r * G::KROW + c;
-    unsigned char* dv = st + G::VOFF + r * G::KROW + c;
-#pragma unroll
-    for (int i = 0; i < kTcTile / 2; ++i)
-      if (2 * i + r < nv) {
-        cp_async16(dk + i * 2 * G::KROW, sk + i * 2 * G::CROW);
-        cp_async16(dv + i * 2 * G::KROW, sv + i * 2 * G::CROW);
-      }
-  } else {
-    // codes: one contiguous block of 16 rows per array; unit u = lane + 32 i
-    constexpr int NI = kTcTile * G::CU / 32;
-    const unsigned char* sk = regk + row0 * G::CROW + lane * 16;
-    const unsigned char* sv = regv + row0 * G::CROW + lane * 16;
-#pragma unroll
-    for (int i = 0; i < NI; ++i)
-      if ((lane + 32 * i) / G::CU < nv) {
-        cp_async16(st + G::KOFF + (lane + 32 * i) * 16, sk + i * 512);
-        cp_async16(st + G::VOFF + (lane + 32 * i) * 16, sv + i * 512);
-      }
-    // scales: one 16-byte row per token; lanes 0-15 K, 16-31 V
-    const int sr = lane & 15;
-    if (sr < nv)
-      cp_async16(st + (lane < 16 ? G::KSOFF : G::VSOFF) + sr * 16,
-                 (lane < 16 ? regk : regv) + soff + (row0 + sr) * 16);
-  }
-  cp_async_commit();
-}
+static_assert(TG<0>::STAGES >= 2 && TG<1>::STAGES >= 3 && TG<2>::STAGES >= 3, "ring too small");
 
 // In-place INT2 code pair at 2-bit position p (0..7) of both 16-bit halves:
 // c * 4^(p or p - 5) * 2^-24 each (positions 5..7 come from x >> 10).
@@ -120,116 +91,141 @@ __device__ __forceinline__ uint32_t nib_at(uint32_t x, uint32_t x8, int n) {
   return (n < 2 ? x : x8) & ((n & 1) ? 0x00F000F0u : 0x000F000Fu);
 }
 
-template <int E>
-__device__ __forceinline__ void tc_item(const unsigned char* __restrict__ regk,
-                                        const unsigned char* __restrict__ regv, uint64_t soff,
-                                        int t0, int n, const __half* __restrict__ q,
-                                        int64_t qbase, float scale_log2, unsigned char* ring,
-                                        int64_t w, float* __restrict__ ws_acc,
-                                        float2* __restrict__ ws_ml) {
+// Copies of one stage: rows [0, nv) of the stage starting at the lane's
+// source pointers (already advanced to the stage's first row).
+template <int E, bool FULL>
+__device__ __forceinline__ void tc_issue(unsigned char* st, const unsigned char* gk,
+                                         const unsigned char* gv, const unsigned char* gks,
+                                         const unsigned char* gvs, int nv, int lane) {
   using G = TG<E>;
-  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-  const int iters = (n + kTcTile - 1) / kTcTile;
-
-#pragma unroll 1
-  for (int s = 0; s < G::STAGES - 1; ++s) {
-    if (s < iters)
-      tc_issue<E>(ring + s * G::STAGE, regk, regv, soff, (int64_t)t0 + s * kTcTile,
-                  min(kTcTile, n - s * kTcTile), lane);
-    else
-      cp_async_commit();
-  }
-
-  // ---- query: one power of two brings max|q| to [2^14, 2^15); per-group sums
-  const __half* qh = q + qbase;
-  float qsa, qsb, qexp;  // sums of groups 2(tig&1), 2(tig&1)+1 (x scale_log2); 2^E
-  {
-    const uint2 raw = *reinterpret_cast<const uint2*>(qh + 4 * lane);
-    const float2 f0 = half2_bits_to_float2(raw.x), f1 = half2_bits_to_float2(raw.y);
-    float mx = fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y)));
-    float sm = (f0.x + f0.y) + (f1.x + f1.y);
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-#pragma unroll
-    for (int off = 1; off < 8; off <<= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
-    const int ga = 2 * (tig & 1);
-    qsa = __shfl_sync(0xffffffffu, sm, 8 * ga) * scale_log2;
-    qsb = __shfl_sync(0xffffffffu, sm, 8 * ga + 8) * scale_log2;
-    const int eb = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;  // floor(log2 max|q|)
-    qexp = mx > 0.f ? __uint_as_float((uint32_t)(127 + 14 - eb) << 23) : 1.f;
-  }
-  // score B operand: qb[ks] for k-step ks
-  uint32_t qb[8][2];
   if constexpr (E == 0) {
-    const bool on = gid == 0;
+    // 16 units per 256-byte row; the lane covers rows r, r + 2, ... at column c
+    const int r = lane >> 4, c = (lane & 15) * 16;
+    unsigned char* dk = st + G::KOFF + r * G::KROW + c;
+    unsigned char* dv = st + G::VOFF + r * G::KROW + c;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const float2 x = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(qh + 16 * ks + 2 * tig));
-      const float2 y = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(qh + 16 * ks + 8 + 2 * tig));
-      const float f = on ? qexp : 0.f;
-      qb[ks][0] = h2_bits(__floats2half2_rn(x.x * f, x.y * f));
-      qb[ks][1] = h2_bits(__floats2half2_rn(y.x * f, y.y * f));
-    }
+    for (int i = 0; i < G::TOK / 2; ++i)
+      if (FULL || 2 * i + r < nv) {
+        cp_async16(dk + i * 2 * G::KROW, gk + i * 2 * G::CROW);
+        cp_async16(dv + i * 2 * G::KROW, gv + i * 2 * G::CROW);
+      }
   } else {
-    const float f = gid == tig ? qexp : 0.f;
-    const __half* qg = qh + 32 * tig;
+    // codes: one contiguous block per array, unit lane + 32 i
+#pragma unroll
+    for (int i = 0; i < G::TOK * G::CU / 32; ++i)
+      if (FULL || (lane + 32 * i) / G::CU < nv) {
+        cp_async16(st + G::KOFF + lane * 16 + i * 512, gk + i * 512);
+        cp_async16(st + G::VOFF + lane * 16 + i * 512, gv + i * 512);
+      }
+    // scales: one 16-byte row per token, row lane
+    if (FULL || lane < nv) {
+      cp_async16(st + G::KSOFF + lane * 16, gks);
+      cp_async16(st + G::VSOFF + lane * 16, gvs);
+    }
+  }
+  cp_async_commit();
+}
+
+// Running state of the item in progress (one query head).
+struct TcState {
+  float o[8][4];
+  float m, m8, l;
+  uint64_t bias2;
+  float down, vlim;  // value unit 2^A as 2^-A and 2^(A+1) (quantised items)
+};
+
+__device__ __forceinline__ void tc_reset(TcState& S) {
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) S.o[mt][0] = S.o[mt][1] = S.o[mt][2] = S.o[mt][3] = 0.f;
+  S.m = -INFINITY;
+  S.m8 = -INFINITY;
+  S.l = 0.f;
+  S.bias2 = 0ull;
+  S.down = 16384.0f;          // A = -14 until a larger scale arrives
+  S.vlim = 1.0f / 8192.0f;
+}
+
+// Per-run query operands and constants.
+struct TcQuery {
+  uint32_t qb[8][2];  // score B operand per k-step
+  float qsa, qsb;     // (scale_log2 x) sums of q over groups 2(tig&1), 2(tig&1)+1
+  float sfac;         // code or fp16 dot -> log2-domain score
+};
+
+template <int E>
+__device__ __forceinline__ void tc_query(TcQuery& Q, const __half* __restrict__ qh, float scale_log2,
+                                         int lane) {
+  const int gid = lane >> 2, tig = lane & 3;
+  // lane holds dims 4 lane .. 4 lane + 3
+  const uint2 raw = *reinterpret_cast<const uint2*>(qh + 4 * lane);
+  const float2 f0 = half2_bits_to_float2(raw.x), f1 = half2_bits_to_float2(raw.y);
+  float mx = fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y)));
+  float sm = (f0.x + f0.y) + (f1.x + f1.y);
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
+  const int ga = 2 * (tig & 1);
+  Q.qsa = __shfl_sync(0xffffffffu, sm, 8 * ga) * scale_log2;
+  Q.qsb = __shfl_sync(0xffffffffu, sm, 8 * ga + 8) * scale_log2;
+  if constexpr (E == 0) {
+    // b0 = q[16 ks + 2 tig, +1], b1 = q[16 ks + 8 + 2 tig, +1] on lanes gid == 0
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      int d0, d1, e0, e1;  // dims of the (b0, b1) pairs; second element of each at +e
-      float c0, c1;        // 1 / position scale of each pair
+      const int l0 = 4 * ks + (tig >> 1), l1 = 4 * ks + 2 + (tig >> 1);
+      const uint32_t x0 = __shfl_sync(0xffffffffu, raw.x, l0), y0 = __shfl_sync(0xffffffffu, raw.y, l0);
+      const uint32_t x1 = __shfl_sync(0xffffffffu, raw.x, l1), y1 = __shfl_sync(0xffffffffu, raw.y, l1);
+      Q.qb[ks][0] = gid == 0 ? ((tig & 1) ? y0 : x0) : 0u;
+      Q.qb[ks][1] = gid == 0 ? ((tig & 1) ? y1 : x1) : 0u;
+    }
+    Q.sfac = scale_log2;
+  } else {
+    // one power of two brings max|q| to [2^14, 2^15)
+    const int eb = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;
+    const float qexp = mx > 0.f ? __uint_as_float((uint32_t)(127 + 14 - eb) << 23) : 1.f;
+    const float f = gid == tig ? qexp : 0.f;  // group tig's column is lane (tig, tig)'s
+    const float qv[4] = {f0.x, f0.y, f1.x, f1.y};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      // dims (d, d + e) of pair b0 and (d1, d1 + e) of b1, inside group tig;
+      // each dim's element index (d mod 4) is the same on every lane
+      int d0, d1, e;
+      float c0, c1;  // 1 / position scale
       if constexpr (E == 1) {
-        d0 = 8 * (ks / 2) + 2 * (ks % 2); d1 = d0 + 1; e0 = e1 = 4;
+        d0 = 8 * (ks / 2) + 2 * (ks % 2); d1 = d0 + 1; e = 4;
         c0 = 1.f; c1 = 1.f / 16.f;
       } else {
-        const int p0 = 2 * (ks % 4), p1 = p0 + 1;
-        d0 = 16 * (ks / 4) + p0; d1 = 16 * (ks / 4) + p1; e0 = e1 = 8;
-        c0 = 1.f / crumb_scale(p0); c1 = 1.f / crumb_scale(p1);
+        const int p0 = 2 * (ks % 4);
+        d0 = 16 * (ks / 4) + p0; d1 = d0 + 1; e = 8;
+        c0 = 1.f / crumb_scale(p0); c1 = 1.f / crumb_scale(p0 + 1);
       }
-      qb[ks][0] = h2_bits(__floats2half2_rn(__half2float(qg[d0]) * f * c0, __half2float(qg[d0 + e0]) * f * c0));
-      qb[ks][1] = h2_bits(__floats2half2_rn(__half2float(qg[d1]) * f * c1, __half2float(qg[d1 + e1]) * f * c1));
+      const int src = 8 * tig;  // lane holding dims 32 tig .. 32 tig + 3
+      const float a0 = __shfl_sync(0xffffffffu, qv[d0 & 3], src + d0 / 4);
+      const float a1 = __shfl_sync(0xffffffffu, qv[d0 & 3], src + (d0 + e) / 4);
+      const float b0 = __shfl_sync(0xffffffffu, qv[d1 & 3], src + d1 / 4);
+      const float b1 = __shfl_sync(0xffffffffu, qv[d1 & 3], src + (d1 + e) / 4);
+      Q.qb[ks][0] = h2_bits(__floats2half2_rn(a0 * f * c0, a1 * f * c0));
+      Q.qb[ks][1] = h2_bits(__floats2half2_rn(b0 * f * c1, b1 * f * c1));
     }
+    // undoes 2^E and the codes' 2^-24
+    Q.sfac = scale_log2 / qexp * 16777216.0f;
   }
-  // score = sfac * (code or fp16 dot) [+ mins]: undoes 2^E and, for codes, the 2^-24
-  const float sfac = scale_log2 / qexp * (E == 0 ? 1.f : 16777216.0f);
+}
 
-  // p redistribution: this lane's B' rows are tokens tau_j; source lanes of each
-  int src[4], tau[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    if constexpr (E == 0) {
-      tau[j] = 2 * tig + (j & 1) + 8 * (j >> 1);
-    } else {
-      tau[j] = tig + 4 * j;
-    }
-    src[j] = 4 * (tau[j] & 7) + (tau[j] >> 3);
-  }
-
-  float o[8][4];
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  float m = -INFINITY, m8 = -INFINITY, l = 0.f;
-  uint64_t bias2 = 0ull;
-  // value unit 2^A (INT tiles): B' = p * s * 2^-A stays below 2^9; A only rises
-  float down = 16384.0f, vlim = 1.0f / 8192.0f;  // A = -14 until a larger scale arrives
+// One stage: scores of its subtiles, online softmax, B', values.
+template <int E, bool FULL>
+__device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const unsigned char* st,
+                                         int nv, int lane) {
+  using G = TG<E>;
+  constexpr int SUB = G::SUB;
+  const int gid = lane >> 2, tig = lane & 3;
   const int g = gid >> 1;
   const bool hl = gid & 1;
 
-#pragma unroll 1
-  for (int it = 0; it < iters; ++it) {
-    {
-      const int nx = it + G::STAGES - 1;
-      if (nx < iters)
-        tc_issue<E>(ring + (nx % G::STAGES) * G::STAGE, regk, regv, soff,
-                    (int64_t)t0 + nx * kTcTile, min(kTcTile, n - nx * kTcTile), lane);
-      else
-        cp_async_commit();
-    }
-    cp_async_wait<G::STAGES - 1>();
-    __syncwarp();
-    unsigned char* st = ring + (it % G::STAGES) * G::STAGE;
-    const int nv = min(kTcTile, n - it * kTcTile);
-
-    // ---- scores (two accumulator chains)
+  // ---- scores of rows gid, gid + 8 of each subtile (two accumulator chains)
+  float sc[SUB][2];
+#pragma unroll
+  for (int u = 0; u < SUB; ++u) {
     float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
     if constexpr (E == 0) {
       const int j = lane >> 3;
@@ -238,174 +234,217 @@ __device__ __forceinline__ void tc_item(const unsigned char* __restrict__ regk,
       for (int ks = 0; ks < 8; ++ks) {
         uint32_t a[4];
         ldsm_x4(a, arow + ks * 32);
-        mma16816(ks < 4 ? c0 : c1, a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+        mma16816(ks < 4 ? c0 : c1, a[0], a[1], a[2], a[3], Q.qb[ks][0], Q.qb[ks][1]);
       }
-    } else if constexpr (E == 1) {
-      const uint4 w0 = *reinterpret_cast<const uint4*>(st + G::KOFF + gid * 64 + 16 * tig);
-      const uint4 w1 = *reinterpret_cast<const uint4*>(st + G::KOFF + (gid + 8) * 64 + 16 * tig);
-      const uint32_t r0[4] = {w0.x, w0.y, w0.z, w0.w}, r1[4] = {w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t x0 = r0[ks / 2], x1 = r1[ks / 2];
-        const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
-        const int nb = 2 * (ks % 2);
-        mma16816(ks < 4 ? c0 : c1, nib_at(x0, y0, nb), nib_at(x1, y1, nb), nib_at(x0, y0, nb + 1),
-                 nib_at(x1, y1, nb + 1), qb[ks][0], qb[ks][1]);
-      }
+      sc[u][0] = ((c0[0] + c1[0]) + (c0[1] + c1[1])) * Q.sfac;
+      sc[u][1] = ((c0[2] + c1[2]) + (c0[3] + c1[3])) * Q.sfac;
     } else {
-      const uint2 w0 = *reinterpret_cast<const uint2*>(st + G::KOFF + gid * 32 + 8 * tig);
-      const uint2 w1 = *reinterpret_cast<const uint2*>(st + G::KOFF + (gid + 8) * 32 + 8 * tig);
-      const uint32_t r0[2] = {w0.x, w0.y}, r1[2] = {w1.x, w1.y};
+      const unsigned char* kr = st + G::KOFF + (16 * u + gid) * G::CROW;
+      if constexpr (E == 1) {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(kr + 16 * tig);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 8 * G::CROW + 16 * tig);
+        const uint32_t r0[4] = {w0.x, w0.y, w0.z, w0.w}, r1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t x0 = r0[ks / 4], x1 = r1[ks / 4];
-        const uint32_t y0 = x0 >> 10, y1 = x1 >> 10;
-        const int p0 = 2 * (ks % 4);
-        mma16816(ks < 4 ? c0 : c1, crumb_at(x0, y0, p0), crumb_at(x1, y1, p0),
-                 crumb_at(x0, y0, p0 + 1), crumb_at(x1, y1, p0 + 1), qb[ks][0], qb[ks][1]);
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t x0 = r0[ks / 2], x1 = r1[ks / 2];
+          const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
+          const int nb = 2 * (ks % 2);
+          mma16816(ks < 4 ? c0 : c1, nib_at(x0, y0, nb), nib_at(x1, y1, nb), nib_at(x0, y0, nb + 1),
+                   nib_at(x1, y1, nb + 1), Q.qb[ks][0], Q.qb[ks][1]);
+        }
+      } else {
+        const uint2 w0 = *reinterpret_cast<const uint2*>(kr + 8 * tig);
+        const uint2 w1 = *reinterpret_cast<const uint2*>(kr + 8 * G::CROW + 8 * tig);
+        const uint32_t r0[2] = {w0.x, w0.y}, r1[2] = {w1.x, w1.y};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t x0 = r0[ks / 4], x1 = r1[ks / 4];
+          const uint32_t y0 = x0 >> 10, y1 = x1 >> 10;
+          const int p0 = 2 * (ks % 4);
+          mma16816(ks < 4 ? c0 : c1, crumb_at(x0, y0, p0), crumb_at(x1, y1, p0),
+                   crumb_at(x0, y0, p0 + 1), crumb_at(x1, y1, p0 + 1), Q.qb[ks][0], Q.qb[ks][1]);
+        }
       }
-    }
-    // this lane's share of the scores of rows gid, gid + 8 (log2 units)
-    float sc0, sc1;
-    if constexpr (E == 0) {
-      sc0 = ((c0[0] + c1[0]) + (c0[1] + c1[1])) * sfac;
-      sc1 = ((c0[2] + c1[2]) + (c0[3] + c1[3])) * sfac;
-    } else {
-      const uint2 k0 = *reinterpret_cast<const uint2*>(st + G::KSOFF + gid * 16 + 8 * (tig & 1));
-      const uint2 k1 = *reinterpret_cast<const uint2*>(st + G::KSOFF + (gid + 8) * 16 + 8 * (tig & 1));
+      const unsigned char* ksr = st + G::KSOFF + (16 * u + gid) * 16 + 8 * (tig & 1);
+      const uint2 k0 = *reinterpret_cast<const uint2*>(ksr);
+      const uint2 k1 = *reinterpret_cast<const uint2*>(ksr + 8 * 16);
       const float2 a0 = half2_bits_to_float2(k0.x), b0 = half2_bits_to_float2(k0.y);
       const float2 a1 = half2_bits_to_float2(k1.x), b1 = half2_bits_to_float2(k1.y);
-      sc0 = fmaf(fmaf(a0.x, c0[0] + c1[0], b0.x * (c0[1] + c1[1])), sfac, fmaf(a0.y, qsa, b0.y * qsb));
-      sc1 = fmaf(fmaf(a1.x, c0[2] + c1[2], b1.x * (c0[3] + c1[3])), sfac, fmaf(a1.y, qsa, b1.y * qsb));
+      sc[u][0] = fmaf(fmaf(a0.x, c0[0] + c1[0], b0.x * (c0[1] + c1[1])), Q.sfac,
+                      fmaf(a0.y, Q.qsa, b0.y * Q.qsb));
+      sc[u][1] = fmaf(fmaf(a1.x, c0[2] + c1[2], b1.x * (c0[3] + c1[3])), Q.sfac,
+                      fmaf(a1.y, Q.qsa, b1.y * Q.qsb));
     }
-    sc0 += __shfl_xor_sync(0xffffffffu, sc0, 1);
-    sc1 += __shfl_xor_sync(0xffffffffu, sc1, 1);
-    // rows past the item's end hold stale bytes (maybe not numbers): masked by
-    // a select; lanes tig >= 2 hold no score
-    const float x0 = (tig < 2 && gid < nv) ? sc0 : -INFINITY;
-    const float x1 = (tig < 2 && gid + 8 < nv) ? sc1 : -INFINITY;
-
-    // ---- online softmax, reference moved lazily (uniform over the warp)
-    if (__any_sync(0xffffffffu, fmaxf(x0, x1) > m8)) {
-      float mx = fmaxf(x0, x1);
+  }
+  // full scores (lanes tig 0, 1); rows past the item's end hold stale bytes
+  // (maybe not numbers) and are masked by a select; lanes tig >= 2 hold none
+  float x[SUB][2];
 #pragma unroll
-      for (int off = 2; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const float a = ex2_ftz(m - mx);
-      m = mx;
-      m8 = mx + kTcRescale;
-      l *= a;
-      bias2 = mul2(bias2, pk2(a, a));
+  for (int u = 0; u < SUB; ++u)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float v = sc[u][r] + __shfl_xor_sync(0xffffffffu, sc[u][r], 1);
+      x[u][r] = (tig < 2 && (FULL || 16 * u + 8 * r + gid < nv)) ? v : -INFINITY;
+    }
+
+  // ---- online softmax, reference moved lazily (uniform over the warp)
+  float mx = fmaxf(x[0][0], x[0][1]);
+  if constexpr (SUB == 2) mx = fmaxf(mx, fmaxf(x[1][0], x[1][1]));
+  if (__any_sync(0xffffffffu, mx > S.m8)) {
+#pragma unroll
+    for (int off = 2; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float a = ex2_ftz(S.m - mx);
+    S.m = mx;
+    S.m8 = mx + kTcRescale;
+    S.l *= a;
+    S.bias2 = mul2(S.bias2, pk2(a, a));
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) S.o[mt][i] *= a;
+  }
+  // this lane's B' rows are tokens tau_j of each subtile: INT tig + 4 j (the
+  // V operand's token pairs), FP16 the ldmatrix order 2 tig + (j & 1) + 8 (j >> 1)
+  float P[SUB][4];
+#pragma unroll
+  for (int u = 0; u < SUB; ++u) {
+    const float p0 = ex2_ftz(x[u][0] - S.m), p1 = ex2_ftz(x[u][1] - S.m);
+    const float pv = (tig & 1) ? p1 : p0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int tau = E == 0 ? 2 * tig + (j & 1) + 8 * (j >> 1) : tig + 4 * j;
+      P[u][j] = __shfl_sync(0xffffffffu, pv, 4 * (tau & 7) + (tau >> 3));
+    }
+    S.l += (P[u][0] + P[u][1]) + (P[u][2] + P[u][3]);
+  }
+
+  // ---- B' = p * s (* 2^-A), high or low fp16 part by column
+  uint32_t bb[SUB][2];
+  if constexpr (E == 0) {
+    const uint32_t h01 = h2_bits(__floats2half2_rn(P[0][0], P[0][1]));
+    const uint32_t h23 = h2_bits(__floats2half2_rn(P[0][2], P[0][3]));
+    const float2 f01 = half2_bits_to_float2(h01), f23 = half2_bits_to_float2(h23);
+    const uint32_t l01 = h2_bits(__floats2half2_rn(P[0][0] - f01.x, P[0][1] - f01.y));
+    const uint32_t l23 = h2_bits(__floats2half2_rn(P[0][2] - f23.x, P[0][3] - f23.y));
+    bb[0][0] = gid >= 2 ? 0u : (hl ? l01 : h01);
+    bb[0][1] = gid >= 2 ? 0u : (hl ? l23 : h23);
+  } else {
+    float vs[SUB][4], vm[SUB][4];
+#pragma unroll
+    for (int u = 0; u < SUB; ++u)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = 16 * u + tig + 4 * j;
+        uint32_t raw = *reinterpret_cast<const uint32_t*>(st + G::VSOFF + row * 16 + 4 * g);
+        if (!FULL) raw = row < nv ? raw : 0u;  // stale scales may not be numbers
+        const float2 f = half2_bits_to_float2(raw);
+        vs[u][j] = f.x;
+        vm[u][j] = f.y;
+      }
+    float vmax = fmaxf(fmaxf(vs[0][0], vs[0][1]), fmaxf(vs[0][2], vs[0][3]));
+    if constexpr (SUB == 2) vmax = fmaxf(vmax, fmaxf(fmaxf(vs[1][0], vs[1][1]), fmaxf(vs[1][2], vs[1][3])));
+    if (__any_sync(0xffffffffu, vmax >= S.vlim)) {
+      float v = vmax;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+      const uint32_t eb = __float_as_uint(v) & 0x7F800000u;     // 2^k, v in [2^k, 2^(k+1))
+      const float dn = __uint_as_float(0x7F000000u - eb);         // 2^-k
+      const float f = dn / S.down;                                 // exact power of two
+      S.down = dn;
+      S.vlim = __uint_as_float(eb + 0x00800000u);                  // 2^(k+1)
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) o[mt][i] *= a;
+        for (int i = 0; i < 4; ++i) S.o[mt][i] *= f;
     }
-    const float p0 = ex2_ftz(x0 - m), p1 = ex2_ftz(x1 - m);
-    const float pv = (tig & 1) ? p1 : p0;
-    float P[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) P[j] = __shfl_sync(0xffffffffu, pv, src[j]);
-    l += (P[0] + P[1]) + (P[2] + P[3]);
-
-    // ---- B' = p * s (* 2^-A), high or low fp16 part by column
-    uint32_t bb0, bb1;
-    if constexpr (E == 0) {
-      const uint32_t h01 = h2_bits(__floats2half2_rn(P[0], P[1]));
-      const uint32_t h23 = h2_bits(__floats2half2_rn(P[2], P[3]));
-      const float2 f01 = half2_bits_to_float2(h01), f23 = half2_bits_to_float2(h23);
-      const uint32_t l01 = h2_bits(__floats2half2_rn(P[0] - f01.x, P[1] - f01.y));
-      const uint32_t l23 = h2_bits(__floats2half2_rn(P[2] - f23.x, P[3] - f23.y));
-      bb0 = gid >= 2 ? 0u : (hl ? l01 : h01);
-      bb1 = gid >= 2 ? 0u : (hl ? l23 : h23);
-    } else {
-      float vs[4], vm[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t raw = *reinterpret_cast<const uint32_t*>(st + G::VSOFF + tau[j] * 16 + 4 * g);
-        const float2 f = half2_bits_to_float2(tau[j] < nv ? raw : 0u);
-        vs[j] = f.x;
-        vm[j] = f.y;
-      }
-      const float vmax = fmaxf(fmaxf(vs[0], vs[1]), fmaxf(vs[2], vs[3]));
-      if (__any_sync(0xffffffffu, vmax >= vlim)) {
-        float mx = vmax;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const uint32_t eb = __float_as_uint(mx) & 0x7F800000u;     // 2^k, mx in [2^k, 2^(k+1))
-        const float dn = __uint_as_float(0x7F000000u - eb);         // 2^-k
-        const float f = dn / down;                                  // exact power of two
-        down = dn;
-        vlim = __uint_as_float(eb + 0x00800000u);                    // 2^(k+1)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[mt][i] *= f;
-      }
-      bias2 = fma2(pk2(P[0], P[1]), pk2(vm[0], vm[1]), bias2);
-      bias2 = fma2(pk2(P[2], P[3]), pk2(vm[2], vm[3]), bias2);
-      const uint64_t w01 = mul2(pk2(P[0] * down, P[1] * down), pk2(vs[0], vs[1]));
-      const uint64_t w23 = mul2(pk2(P[2] * down, P[3] * down), pk2(vs[2], vs[3]));
+    for (int u = 0; u < SUB; ++u) {
+      S.bias2 = fma2(pk2(P[u][0], P[u][1]), pk2(vm[u][0], vm[u][1]), S.bias2);
+      S.bias2 = fma2(pk2(P[u][2], P[u][3]), pk2(vm[u][2], vm[u][3]), S.bias2);
+      const uint64_t dn2 = pk2(S.down, S.down);
+      const uint64_t w01 = mul2(mul2(pk2(P[u][0], P[u][1]), dn2), pk2(vs[u][0], vs[u][1]));
+      const uint64_t w23 = mul2(mul2(pk2(P[u][2], P[u][3]), dn2), pk2(vs[u][2], vs[u][3]));
       const uint32_t h01 = h2_bits(__floats2half2_rn(lo2(w01), hi2(w01)));
       const uint32_t h23 = h2_bits(__floats2half2_rn(lo2(w23), hi2(w23)));
       const float2 f01 = half2_bits_to_float2(h01), f23 = half2_bits_to_float2(h23);
       const uint64_t r01 = sub2(w01, pk2(f01.x, f01.y)), r23 = sub2(w23, pk2(f23.x, f23.y));
       const uint32_t l01 = h2_bits(__floats2half2_rn(lo2(r01), hi2(r01)));
       const uint32_t l23 = h2_bits(__floats2half2_rn(lo2(r23), hi2(r23)));
-      bb0 = hl ? l01 : h01;
-      bb1 = hl ? l23 : h23;
+      bb[u][0] = hl ? l01 : h01;
+      bb[u][1] = hl ? l23 : h23;
     }
+  }
 
-    // ---- values
-    if constexpr (E == 0) {
-      if (nv < kTcTile) {  // stale rows may not be numbers, and 0 * NaN is NaN
-        constexpr int RU = 256 / 16;
-        for (int u = lane; u < (kTcTile - nv) * RU; u += 32)
-          *reinterpret_cast<uint4*>(st + G::VOFF + (nv + u / RU) * G::KROW + (u % RU) * 16) =
-              make_uint4(0, 0, 0, 0);
-        __syncwarp();
-      }
-      const int j = lane >> 3;
-      const uint32_t arow = smem_addr(st + G::VOFF) + ((lane & 7) + (j >> 1) * 8) * G::KROW + (j & 1) * 16;
+  // ---- values: O^T += Vhat^T . B'
+  if constexpr (E == 0) {
+    unsigned char* stw = const_cast<unsigned char*>(st);
+    if (!FULL) {  // stale rows may not be numbers, and 0 * NaN is NaN
+      constexpr int RU = 256 / 16;
+      for (int i = lane; i < (16 - nv) * RU; i += 32)
+        *reinterpret_cast<uint4*>(stw + G::VOFF + (nv + i / RU) * G::KROW + (i % RU) * 16) =
+            make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
+    const int j = lane >> 3;
+    const uint32_t arow = smem_addr(st + G::VOFF) + ((lane & 7) + (j >> 1) * 8) * G::KROW + (j & 1) * 16;
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t a[4];
-        ldsm_x4_t(a, arow + mt * 32);
-        mma16816(o[mt], a[0], a[1], a[2], a[3], bb0, bb1);
-      }
-    } else if constexpr (E == 1) {
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_t(a, arow + mt * 32);
+      mma16816(S.o[mt], a[0], a[1], a[2], a[3], bb[0][0], bb[0][1]);
+    }
+  } else if constexpr (E == 1) {
+    uint32_t la01[SUB], ha01[SUB], lb01[SUB], hb01[SUB], la23[SUB], ha23[SUB], lb23[SUB], hb23[SUB];
+#pragma unroll
+    for (int u = 0; u < SUB; ++u) {
       uint2 v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint2*>(st + G::VOFF + tau[j] * 64 + 8 * gid);
+      for (int jj = 0; jj < 4; ++jj)
+        v[jj] = *reinterpret_cast<const uint2*>(st + G::VOFF + (16 * u + tig + 4 * jj) * 64 + 8 * gid);
       // halves of token pairs (0, 1) and (2, 3): dims 0-3, 4-7 (word a), 8-11, 12-15 (word b)
-      const uint32_t la01 = __byte_perm(v[0].x, v[1].x, 0x5410), ha01 = __byte_perm(v[0].x, v[1].x, 0x7632);
-      const uint32_t lb01 = __byte_perm(v[0].y, v[1].y, 0x5410), hb01 = __byte_perm(v[0].y, v[1].y, 0x7632);
-      const uint32_t la23 = __byte_perm(v[2].x, v[3].x, 0x5410), ha23 = __byte_perm(v[2].x, v[3].x, 0x7632);
-      const uint32_t lb23 = __byte_perm(v[2].y, v[3].y, 0x5410), hb23 = __byte_perm(v[2].y, v[3].y, 0x7632);
+      la01[u] = __byte_perm(v[0].x, v[1].x, 0x5410); ha01[u] = __byte_perm(v[0].x, v[1].x, 0x7632);
+      lb01[u] = __byte_perm(v[0].y, v[1].y, 0x5410); hb01[u] = __byte_perm(v[0].y, v[1].y, 0x7632);
+      la23[u] = __byte_perm(v[2].x, v[3].x, 0x5410); ha23[u] = __byte_perm(v[2].x, v[3].x, 0x7632);
+      lb23[u] = __byte_perm(v[2].y, v[3].y, 0x5410); hb23[u] = __byte_perm(v[2].y, v[3].y, 0x7632);
+    }
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const uint32_t xa01 = mt < 4 ? la01 : ha01, xb01 = mt < 4 ? lb01 : hb01;
-        const uint32_t xa23 = mt < 4 ? la23 : ha23, xb23 = mt < 4 ? lb23 : hb23;
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int u = 0; u < SUB; ++u) {
+        const uint32_t xa01 = mt < 4 ? la01[u] : ha01[u], xb01 = mt < 4 ? lb01[u] : hb01[u];
+        const uint32_t xa23 = mt < 4 ? la23[u] : ha23[u], xb23 = mt < 4 ? lb23[u] : hb23[u];
         const int nb = mt & 3;
-        mma16816(o[mt], nib_at(xa01, xa01 >> 8, nb), nib_at(xb01, xb01 >> 8, nb),
-                 nib_at(xa23, xa23 >> 8, nb), nib_at(xb23, xb23 >> 8, nb), bb0, bb1);
+        mma16816(S.o[mt], nib_at(xa01, xa01 >> 8, nb), nib_at(xb01, xb01 >> 8, nb),
+                 nib_at(xa23, xa23 >> 8, nb), nib_at(xb23, xb23 >> 8, nb), bb[u][0], bb[u][1]);
       }
-    } else {
+  } else {
+    uint32_t l01[SUB], h01[SUB], l23[SUB], h23[SUB];
+#pragma unroll
+    for (int u = 0; u < SUB; ++u) {
       uint32_t v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint32_t*>(st + G::VOFF + tau[j] * 32 + 4 * gid);
-      const uint32_t l01 = __byte_perm(v[0], v[1], 0x5410), h01 = __byte_perm(v[0], v[1], 0x7632);
-      const uint32_t l23 = __byte_perm(v[2], v[3], 0x5410), h23 = __byte_perm(v[2], v[3], 0x7632);
-      const uint32_t l01s = l01 >> 10, h01s = h01 >> 10, l23s = l23 >> 10, h23s = h23 >> 10;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
-        mma16816(o[mt], crumb_at(l01, l01s, mt), crumb_at(h01, h01s, mt), crumb_at(l23, l23s, mt),
-                 crumb_at(h23, h23s, mt), bb0, bb1);
+      for (int jj = 0; jj < 4; ++jj)
+        v[jj] = *reinterpret_cast<const uint32_t*>(st + G::VOFF + (16 * u + tig + 4 * jj) * 32 + 4 * gid);
+      l01[u] = __byte_perm(v[0], v[1], 0x5410); h01[u] = __byte_perm(v[0], v[1], 0x7632);
+      l23[u] = __byte_perm(v[2], v[3], 0x5410); h23[u] = __byte_perm(v[2], v[3], 0x7632);
     }
-    __syncwarp();  // the stage is read before it is refilled
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int u = 0; u < SUB; ++u)
+        mma16816(S.o[mt], crumb_at(l01[u], l01[u] >> 10, mt), crumb_at(h01[u], h01[u] >> 10, mt),
+                 crumb_at(l23[u], l23[u] >> 10, mt), crumb_at(h23[u], h23[u] >> 10, mt), bb[u][0],
+                 bb[u][1]);
   }
-  cp_async_wait<0>();
+}
 
-  // ---- partial results of the item
+// Partial record of a finished item: unnormalised accumulator (with the
+// mins' contribution) and (m, l).
+template <int E>
+__device__ __forceinline__ void tc_record(const TcState& S, int lane, int64_t w,
+                                          float* __restrict__ ws_acc, float2* __restrict__ ws_ml) {
+  const int gid = lane >> 2, tig = lane & 3;
+  float l = S.l;
   l += __shfl_xor_sync(0xffffffffu, l, 1);
   l += __shfl_xor_sync(0xffffffffu, l, 2);
   float* dst = ws_acc + (size_t)w * 128;
@@ -414,24 +453,24 @@ __device__ __forceinline__ void tc_item(const unsigned char* __restrict__ regk,
     if (tig == 0) {
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        dst[16 * mt + gid] = o[mt][0] + o[mt][1];
-        dst[16 * mt + gid + 8] = o[mt][2] + o[mt][3];
+        dst[16 * mt + gid] = S.o[mt][0] + S.o[mt][1];
+        dst[16 * mt + gid + 8] = S.o[mt][2] + S.o[mt][3];
       }
     }
   } else {
-    float bias = lo2(bias2) + hi2(bias2);
+    float bias = lo2(S.bias2) + hi2(S.bias2);
     bias += __shfl_xor_sync(0xffffffffu, bias, 1);
     bias += __shfl_xor_sync(0xffffffffu, bias, 2);
     // lanes whose columns (2 tig, 2 tig + 1) are their own dims' group hold
     // dims 16 gid + mt (row gid) and 16 gid + 8 + mt (row gid + 8)
-    if (tig == g) {
-      const float up = 16777216.0f / down;  // 2^A and the codes' 2^-24
+    if (tig == (gid >> 1)) {
+      const float up = 16777216.0f / S.down;  // 2^A and the codes' 2^-24
       float r0[8], r1[8];
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
         const float f = up / (E == 1 ? ((mt & 1) ? 16.f : 1.f) : crumb_scale(mt));
-        r0[mt] = fmaf(o[mt][0] + o[mt][1], f, bias);
-        r1[mt] = fmaf(o[mt][2] + o[mt][3], f, bias);
+        r0[mt] = fmaf(S.o[mt][0] + S.o[mt][1], f, bias);
+        r1[mt] = fmaf(S.o[mt][2] + S.o[mt][3], f, bias);
       }
       float4* d4 = reinterpret_cast<float4*>(dst + 16 * gid);
       d4[0] = make_float4(r0[0], r0[1], r0[2], r0[3]);
@@ -440,7 +479,84 @@ __device__ __forceinline__ void tc_item(const unsigned char* __restrict__ regk,
       d4[3] = make_float4(r1[4], r1[5], r1[6], r1[7]);
     }
   }
-  if (lane == 0) ws_ml[w] = make_float2(m, l);
+  if (lane == 0) ws_ml[w] = make_float2(S.m, l);
+}
+
+// One run: tokens [T0, T1) of one region (the region's items j0, j0 + 1, ...
+// of IT tokens each; records w0, w0 + Hkv, ...), streamed through the ring.
+template <int E>
+__device__ __forceinline__ void tc_run(const unsigned char* __restrict__ regk,
+                                       const unsigned char* __restrict__ regv, uint64_t soff,
+                                       int T0, int T1, int IT, int64_t w0, int Hkv,
+                                       const __half* __restrict__ qh, float scale_log2,
+                                       unsigned char* ring, float* __restrict__ ws_acc,
+                                       float2* __restrict__ ws_ml) {
+  using G = TG<E>;
+  const int lane = threadIdx.x & 31;
+  const int ntok = T1 - T0;
+  const int nst = (ntok + G::TOK - 1) / G::TOK;
+
+  // the lane's copy sources at the run's first stage; each stage advances them
+  const unsigned char *gk, *gv, *gks = nullptr, *gvs = nullptr;
+  if constexpr (E == 0) {
+    const int64_t row = (int64_t)T0 + (lane >> 4);
+    gk = regk + row * G::CROW + (lane & 15) * 16;
+    gv = regv + row * G::CROW + (lane & 15) * 16;
+  } else {
+    gk = regk + (int64_t)T0 * G::CROW + lane * 16;
+    gv = regv + (int64_t)T0 * G::CROW + lane * 16;
+    gks = regk + soff + ((int64_t)T0 + lane) * 16;
+    gvs = regv + soff + ((int64_t)T0 + lane) * 16;
+  }
+  constexpr int CSTEP = G::TOK * G::CROW, SSTEP = G::TOK * 16;
+  int issued = 0;
+  auto issue_next = [&]() {
+    if (issued < nst) {
+      unsigned char* st = ring + (issued % G::STAGES) * G::STAGE;
+      const int nv = min(G::TOK, ntok - issued * G::TOK);
+      if (nv == G::TOK)
+        tc_issue<E, true>(st, gk, gv, gks, gvs, nv, lane);
+      else
+        tc_issue<E, false>(st, gk, gv, gks, gvs, nv, lane);
+      gk += CSTEP;
+      gv += CSTEP;
+      if constexpr (E != 0) {
+        gks += SSTEP;
+        gvs += SSTEP;
+      }
+    } else {
+      cp_async_commit();
+    }
+    ++issued;
+  };
+#pragma unroll 1
+  for (int s = 0; s < G::STAGES - 1; ++s) issue_next();
+
+  TcQuery Q;
+  tc_query<E>(Q, qh, scale_log2, lane);
+  TcState S;
+  tc_reset(S);
+  int64_t w = w0;
+
+#pragma unroll 1
+  for (int k = 0; k < nst; ++k) {
+    issue_next();
+    cp_async_wait<G::STAGES - 1>();
+    __syncwarp();
+    const unsigned char* st = ring + (k % G::STAGES) * G::STAGE;
+    const int nv = min(G::TOK, ntok - k * G::TOK);
+    if (nv == G::TOK)
+      tc_stage<E, true>(S, Q, st, nv, lane);
+    else
+      tc_stage<E, false>(S, Q, st, nv, lane);
+    if (((k + 1) * G::TOK) % IT == 0 || k == nst - 1) {
+      tc_record<E>(S, lane, w, ws_acc, ws_ml);
+      tc_reset(S);
+      w += Hkv;
+    }
+    __syncwarp();  // the stage is read before it is refilled
+  }
+  cp_async_wait<0>();
   __syncwarp();
 }
 
@@ -462,34 +578,55 @@ decode_mha_kernel(const unsigned char* __restrict__ layout, const unsigned char*
     return;
   }
   const int lane = threadIdx.x & 31;
+  const int64_t workers = (int64_t)gridDim.x;
+  // Items in region order: v = Hkv * item_begin[s] + g * item_count[s] + j for
+  // item j of segment s, kv-head g of a sequence (its record is
+  // (item_begin[s] + j) * Hkv + g).
   for (;;) {
-    unsigned int wi = 0;
-    if (lane == 0) wi = atomicAdd(counter, 1u);
-    const int64_t w = (int64_t)__shfl_sync(0xffffffffu, wi, 0);
-    if (w >= total) break;
-    const int64_t bs = w / Hkv;
-    const int g = (int)(w - bs * Hkv);
-    const int b = find_item_seq(layout, B, bs);
-    const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
-    const int s = bs < r->item_begin[1] ? 0 : (bs < r->item_begin[2] ? 1 : 2);
-    const int j = (int)(bs - r->item_begin[s]);
-    const int t0 = j * h->item_tokens[s];
-    const int n = min(h->item_tokens[s], r->seg_tokens[s] - t0);
-    if (n <= 0) {
-      if (lane == 0) set_status(status, MQ_DEV_INDEX_RANGE);
-      continue;
+    // guided claim: a group of up to kTcMaxGroup items, about the remaining
+    // work over twice the workers
+    unsigned int v0 = 0, cnt = 0;
+    if (lane == 0) {
+      const int64_t cur = (int64_t)*reinterpret_cast<volatile unsigned int*>(counter);
+      const int64_t want = (total - cur) / (2 * workers);
+      cnt = (unsigned int)(want < 1 ? 1 : (want > kTcMaxGroup ? kTcMaxGroup : want));
+      v0 = atomicAdd(counter, cnt);
     }
-    const unsigned char* regk = packed + r->seg_base[s] + (uint64_t)g * r->region_bytes[s];
-    const unsigned char* regv = regk + (uint64_t)Hkv * r->region_bytes[s];
-    const int64_t qbase = ((int64_t)b * Hkv + g) * 128;
-    if (s == 0)
-      tc_item<0>(regk, regv, 0, t0, n, q, qbase, scale_log2, smem_raw, w, ws_acc, ws_ml);
-    else if (s == 1)
-      tc_item<1>(regk, regv, r->scale_offset[1], t0, n, q, qbase, scale_log2, smem_raw, w, ws_acc,
-                 ws_ml);
-    else
-      tc_item<2>(regk, regv, r->scale_offset[2], t0, n, q, qbase, scale_log2, smem_raw, w, ws_acc,
-                 ws_ml);
+    v0 = __shfl_sync(0xffffffffu, v0, 0);
+    cnt = __shfl_sync(0xffffffffu, cnt, 0);
+    if ((int64_t)v0 >= total) break;
+    const int64_t v1 = min((int64_t)v0 + cnt, total);
+    for (int64_t v = v0; v < v1;) {
+      const int b = find_item_seq(layout, B, v / Hkv);
+      const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
+      const int s = v < (int64_t)Hkv * r->item_begin[1] ? 0 : (v < (int64_t)Hkv * r->item_begin[2] ? 1 : 2);
+      const int64_t base = (int64_t)Hkv * r->item_begin[s];
+      const int cntr = r->item_count[s];
+      const int64_t u = v - base;
+      const int g = cntr > 0 ? (int)(u / cntr) : 0;
+      const int j = cntr > 0 ? (int)(u - (int64_t)g * cntr) : 0;
+      const int64_t vend = min(v1, base + (int64_t)(g + 1) * cntr);  // end of this region's items
+      const int IT = h->item_tokens[s];
+      const int T0 = j * IT;
+      const int T1 = (int)min((int64_t)r->seg_tokens[s], (int64_t)(j + (vend - v)) * IT);
+      if (cntr <= 0 || g >= Hkv || T1 <= T0) {
+        if (lane == 0) set_status(status, MQ_DEV_INDEX_RANGE);
+        break;
+      }
+      const unsigned char* regk = packed + r->seg_base[s] + (uint64_t)g * r->region_bytes[s];
+      const unsigned char* regv = regk + (uint64_t)Hkv * r->region_bytes[s];
+      const int64_t w0 = ((int64_t)r->item_begin[s] + j) * Hkv + g;
+      const __half* qh = q + ((int64_t)b * Hkv + g) * 128;
+      if (s == 0)
+        tc_run<0>(regk, regv, 0, T0, T1, IT, w0, Hkv, qh, scale_log2, smem_raw, ws_acc, ws_ml);
+      else if (s == 1)
+        tc_run<1>(regk, regv, r->scale_offset[1], T0, T1, IT, w0, Hkv, qh, scale_log2, smem_raw,
+                  ws_acc, ws_ml);
+      else
+        tc_run<2>(regk, regv, r->scale_offset[2], T0, T1, IT, w0, Hkv, qh, scale_log2, smem_raw,
+                  ws_acc, ws_ml);
+      v = vend;
+    }
   }
 }
 
