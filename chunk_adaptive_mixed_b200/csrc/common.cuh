@@ -15,6 +15,8 @@ namespace mqkv {
 
 constexpr int kNumExperts = 3;
 constexpr int kGroup = 32;
+// merge slices per (sequence, query head) in the decode combine, at most
+constexpr int kSplitMax = 8;
 
 __host__ __device__ constexpr int expert_bits(int e) { return e == 0 ? 16 : (e == 1 ? 4 : 2); }
 
@@ -146,8 +148,13 @@ cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layo
 // CUDA-core kernel; the counter is zeroed on the stream first.
 cudaError_t launch_decode_mha(int64_t capacity_items, const unsigned char* layout,
                               const unsigned char* packed, const __half* q, float scale_log2,
-                              float* ws_acc, float2* ws_ml, unsigned int* counter,
+                              float* ws_acc, float2* ws_ml, unsigned int* counter, int* tab, int B, int Hq,
                               unsigned int* status, cudaStream_t stream);
+// The same for four query heads per kv-head (decode_gqa.cu).
+cudaError_t launch_decode_gqa4(int64_t capacity_items, const unsigned char* layout,
+                               const unsigned char* packed, const __half* q, float scale_log2,
+                               float* ws_acc, float2* ws_ml, unsigned int* counter, int* tab, int B, int Hq,
+                               unsigned int* status, cudaStream_t stream);
 cudaError_t launch_combine_partials(int P, int B, int Hq, int D, const float* parts, float* out,
                                     cudaStream_t stream);
 

@@ -522,15 +522,22 @@ decode_partial_kernel(const unsigned char* __restrict__ layout,
 // shard: [o (D values, normalised), m, l, 0, 0] with m the reference score of
 // the merged softmax (natural-log units, within 8 ln 2 below the largest
 // score) and l = sum exp(score - m) (mq_decode_attn_partial).
-template <int D, int QPG, bool PARTIAL>
-__global__ void __launch_bounds__(256)
+// Long sequences are split: gridDim.y = S CTAs per (b, h) each merge a fixed
+// slice of the items into a split record [num (D values), M, L] in `split`;
+// the CTA that finishes last (a counter per (b, h) in `done`, zero on entry
+// and left at zero) merges the S records in slice order and writes the
+// output, so the result does not depend on the CTAs' timing.
+template <int D, int QPG, bool PARTIAL, int NW>
+__global__ void __launch_bounds__(32 * NW)
 decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
                       const float* __restrict__ ws_acc, const float2* __restrict__ ws_ml,
-                      float* __restrict__ out) {
+                      float* __restrict__ out, float* __restrict__ split,
+                      unsigned int* __restrict__ done) {
   constexpr int PER_LANE = D / 32;
-  constexpr int NW = 8;
   __shared__ float s_acc[NW][D];
   __shared__ float s_m[NW], s_l[NW];
+  __shared__ int s_last;
+  const int S = gridDim.y, k = blockIdx.y;
   const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
   const int Hkv = h->num_kv_heads;
   const int64_t bh = blockIdx.x;
@@ -538,8 +545,9 @@ decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
   const int g = hq / QPG, hh = hq % QPG;
   const int lane = threadIdx.x & 31, warp = threadIdx.x / 32;
   const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
-  const int i0 = r->item_begin[0];
-  const int i1 = r->item_begin[2] + r->item_count[2];
+  const int n_items = r->item_begin[2] + r->item_count[2] - r->item_begin[0];
+  const int i0 = r->item_begin[0] + (int)((int64_t)n_items * k / S);
+  const int i1 = r->item_begin[0] + (int)((int64_t)n_items * (k + 1) / S);
   float M = -INFINITY, l = 0.f, acc[PER_LANE];
 #pragma unroll
   for (int i = 0; i < PER_LANE; ++i) acc[i] = 0.f;
@@ -587,17 +595,46 @@ decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
     s_l[warp] = l;
   }
   __syncthreads();
+  float Mx = -INFINITY, num = 0.f, den = 0.f;
   if (threadIdx.x < D) {
-    float Mx = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, s_m[w]);
-    float num = 0.f, den = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const float f = s_m[w] == -INFINITY ? 0.f : exp2f(s_m[w] - Mx);
       num += f * s_acc[w][threadIdx.x];
       den += f * s_l[w];
     }
+  }
+  if (S > 1) {
+    // this slice's record, then the last slice's CTA merges all of them
+    float* rec = split + ((size_t)bh * S + k) * (D + 2);
+    if (threadIdx.x < D) rec[threadIdx.x] = num;
+    if (threadIdx.x == 0) {
+      rec[D] = Mx;
+      rec[D + 1] = den;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(done + bh, 1u) == (unsigned int)(S - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (threadIdx.x == 0) done[bh] = 0u;  // ready for the next call
+    Mx = -INFINITY;
+    num = den = 0.f;
+    if (threadIdx.x < D) {
+      const volatile float* base = split + (size_t)bh * S * (D + 2);
+      for (int j = 0; j < S; ++j) Mx = fmaxf(Mx, base[j * (D + 2) + D]);
+      for (int j = 0; j < S; ++j) {
+        const float mj = base[j * (D + 2) + D];
+        const float f = mj == -INFINITY ? 0.f : exp2f(mj - Mx);
+        num += f * base[j * (D + 2) + threadIdx.x];
+        den += f * base[j * (D + 2) + D + 1];
+      }
+    }
+  }
+  if (threadIdx.x < D) {
     if constexpr (PARTIAL) {
       float* rec = out + bh * (D + 4);
       rec[threadIdx.x] = den > 0.f ? num / den : 0.f;
@@ -1155,8 +1192,8 @@ template <int D, int QPG, int QDT>
 cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layout,
                             const unsigned char* packed, const void* q, float scale_log2,
                             float* out, float* ws_acc, float2* ws_ml, unsigned int* counter,
-                            int num_seqs, unsigned int* status, cudaStream_t stream,
-                            bool partial) {
+                            unsigned int* done, int* tab, float* split, int num_seqs,
+                            unsigned int* status, cudaStream_t stream, bool partial) {
   // several query heads per kv-head with fp16 queries: the tensor-core kernel
   constexpr bool kMma = QDT == MQ_F16 && QPG >= 2;
   constexpr size_t smem = kMma ? mma_smem_bytes<D>() : decode_smem_bytes<D, QPG>();
@@ -1176,8 +1213,11 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
     const int64_t need = (cap + warps - 1) / warps;
     if (grid > need) grid = need;
     if (grid > 0) {
-      // worker warps take items from a counter in the workspace, zeroed here
-      if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned int), stream)) != cudaSuccess) return e;
+      // worker warps take items from a counter in the workspace; it and the
+      // merge counters after it start at zero
+      if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned int) * (1 + (size_t)num_seqs * Hq), stream)) !=
+          cudaSuccess)
+        return e;
       kern<<<(unsigned)grid, threads, smem, stream>>>(layout, packed, qptr, scale_log2, ws_acc, ws_ml,
                                                       counter, cap, status);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1186,32 +1226,40 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
   };
   if constexpr (D == 128 && QPG == 1 && QDT == MQ_F16)
     err = launch_decode_mha(cap, layout, packed, static_cast<const __half*>(q), scale_log2, ws_acc,
-                            ws_ml, counter, status, stream);
+                            ws_ml, counter, tab, num_seqs, Hq, status, stream);
+  else if constexpr (D == 128 && QPG == 4 && QDT == MQ_F16)
+    err = launch_decode_gqa4(cap, layout, packed, static_cast<const __half*>(q), scale_log2, ws_acc,
+                             ws_ml, counter, tab, num_seqs, Hq, status, stream);
   else if constexpr (kMma)
     err = run(decode_mma_kernel<D, QPG>, static_cast<const __half*>(q));
   else
     err = run(decode_partial_kernel<D, QPG, QDT>, q);
   if (err != cudaSuccess) return err;
   const int64_t heads = (int64_t)num_seqs * Hq;
+  // long sequences are merged in up to kSplitMax slices of about 64 items
+  const int64_t avg = max_items / Hq * QPG / (num_seqs > 0 ? num_seqs : 1);  // items per (b, h)
+  const int S = (int)(avg / 64 < 1 ? 1 : (avg / 64 > kSplitMax ? kSplitMax : avg / 64));
+  const dim3 grid((unsigned)heads, (unsigned)S);
   if (partial)
-    decode_combine_kernel<D, QPG, true><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc,
-                                                                             ws_ml, out);
+    decode_combine_kernel<D, QPG, true, 8><<<grid, 256, 0, stream>>>(layout, Hq, ws_acc, ws_ml, out,
+                                                                     split, done);
   else
-    decode_combine_kernel<D, QPG, false><<<(unsigned)heads, 256, 0, stream>>>(layout, Hq, ws_acc,
-                                                                              ws_ml, out);
+    decode_combine_kernel<D, QPG, false, 8><<<grid, 256, 0, stream>>>(layout, Hq, ws_acc, ws_ml, out,
+                                                                      split, done);
   return cudaGetLastError();
 }
 
 template <int D, int QDT>
 cudaError_t dispatch_qpg(int qpg, int64_t max_items, int Hq, const unsigned char* layout,
                          const unsigned char* packed, const void* q, float scale_log2, float* out,
-                         float* ws_acc, float2* ws_ml, unsigned int* counter, int B,
-                         unsigned int* status, cudaStream_t stream, bool partial) {
+                         float* ws_acc, float2* ws_ml, unsigned int* counter, unsigned int* done,
+                         int* tab, float* split, int B, unsigned int* status, cudaStream_t stream,
+                         bool partial) {
   switch (qpg) {
-    case 1: return launch_decode_t<D, 1, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
-    case 2: return launch_decode_t<D, 2, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
-    case 4: return launch_decode_t<D, 4, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
-    case 8: return launch_decode_t<D, 8, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, B, status, stream, partial);
+    case 1: return launch_decode_t<D, 1, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, B, status, stream, partial);
+    case 2: return launch_decode_t<D, 2, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, B, status, stream, partial);
+    case 4: return launch_decode_t<D, 4, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, B, status, stream, partial);
+    case 8: return launch_decode_t<D, 8, QDT>(max_items, Hq, layout, packed, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, B, status, stream, partial);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1221,9 +1269,13 @@ cudaError_t dispatch_qpg(int qpg, int64_t max_items, int Hq, const unsigned char
 size_t decode_workspace_bytes(const mq_shape& s, int64_t max_items) {
   const int64_t qpg = s.num_q_heads / s.num_kv_heads;
   const int64_t recs = max_items * s.num_kv_heads * qpg;
-  // partial (acc) records, (m, l) records, the work counter
+  // partial (acc) records, (m, l) records, control words (the work counter,
+  // then one merge counter per (b, h)), the work-order prefix table of the
+  // tensor-core kernels (3 x (B + 1) int32), the merge slices
+  const uint64_t heads = (uint64_t)s.num_seqs * s.num_q_heads;
   return (size_t)align128((uint64_t)recs * s.head_dim * 4) + (size_t)align128((uint64_t)recs * 8) +
-         128;
+         (size_t)align128(4 + heads * 4) + (size_t)align128((uint64_t)3 * (s.num_seqs + 1) * 4) +
+         (size_t)align128(heads * kSplitMax * (s.head_dim + 2) * 4);
 }
 
 cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layout,
@@ -1239,18 +1291,23 @@ cudaError_t launch_decode(const mq_shape& s, int64_t max_items, const void* layo
   unsigned int* counter = reinterpret_cast<unsigned int*>(
       static_cast<unsigned char*>(workspace) + align128((uint64_t)recs * s.head_dim * 4) +
       align128((uint64_t)recs * 8));
+  const uint64_t heads = (uint64_t)s.num_seqs * s.num_q_heads;
+  unsigned int* done = counter + 1;  // merge counters, zeroed with the work counter
+  int* tab = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(counter) + align128(4 + heads * 4));
+  float* split = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(tab) +
+                                          align128((uint64_t)3 * (s.num_seqs + 1) * 4));
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   const unsigned char* lay = static_cast<const unsigned char*>(layout);
   const unsigned char* pk = static_cast<const unsigned char*>(packed);
   const int64_t cap = max_items * s.num_kv_heads;
   if (s.head_dim == 128) {
     if (q_dtype == MQ_F16)
-      return dispatch_qpg<128, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
-    return dispatch_qpg<128, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
+      return dispatch_qpg<128, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, s.num_seqs, status, stream, partial);
+    return dispatch_qpg<128, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, s.num_seqs, status, stream, partial);
   }
   if (q_dtype == MQ_F16)
-    return dispatch_qpg<64, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
-  return dispatch_qpg<64, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, s.num_seqs, status, stream, partial);
+    return dispatch_qpg<64, MQ_F16>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, s.num_seqs, status, stream, partial);
+  return dispatch_qpg<64, MQ_F32>((int)qpg, cap, s.num_q_heads, lay, pk, q, scale_log2, out, ws_acc, ws_ml, counter, done, tab, split, s.num_seqs, status, stream, partial);
 }
 
 cudaError_t launch_combine_partials(int P, int B, int Hq, int D, const float* parts, float* out,

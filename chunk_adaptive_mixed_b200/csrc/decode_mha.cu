@@ -49,82 +49,10 @@
 // took it or on the grouping.  Quantised stages are laid out so that every
 // lane's shared-memory reads are conflict-free without padding; FP16 rows are
 // padded for ldmatrix.
-#include "decode_ptx.cuh"
+#include "decode_tc.cuh"
 
 namespace mqkv {
 namespace {
-
-constexpr int kTcRing = 17408;      // shared bytes per worker warp
-constexpr int kTcCtasPerSm = 12;    // one-warp CTAs resident per SM
-constexpr float kTcRescale = 8.0f;  // lazy softmax reference: weights stay below 2^8
-constexpr int kTcMaxGroup = 8;      // items per claim at most
-
-template <int E>
-struct TG {  // stage geometry at head_dim 128
-  static constexpr int BITS = E == 0 ? 16 : (E == 1 ? 4 : 2);
-  static constexpr int SUB = E == 0 ? 1 : 2;             // 16-token subtiles per stage
-  static constexpr int TOK = 16 * SUB;                   // tokens per stage
-  static constexpr int CROW = 128 * BITS / 8;            // code bytes of a token row
-  static constexpr int KROW = E == 0 ? CROW + 16 : CROW; // staged pitch
-  static constexpr int SROW = E == 0 ? 0 : 16;           // (scale, min) bytes of a row
-  static constexpr int KOFF = 0;
-  static constexpr int VOFF = TOK * KROW;
-  static constexpr int KSOFF = 2 * TOK * KROW;
-  static constexpr int VSOFF = KSOFF + TOK * SROW;
-  static constexpr int STAGE = VSOFF + TOK * SROW;
-  static constexpr int STAGES = kTcRing / STAGE < 8 ? kTcRing / STAGE : 8;
-  static constexpr int CU = CROW / 16;                   // 16-byte units per code row
-};
-static_assert(TG<0>::STAGES >= 2 && TG<1>::STAGES >= 3 && TG<2>::STAGES >= 3, "ring too small");
-
-// In-place INT2 code pair at 2-bit position p (0..7) of both 16-bit halves:
-// c * 4^(p or p - 5) * 2^-24 each (positions 5..7 come from x >> 10).
-__device__ __forceinline__ uint32_t crumb_at(uint32_t x, uint32_t x10, int p) {
-  return p <= 4 ? (x & (0x00030003u << (2 * p))) : (x10 & (0x00030003u << (2 * (p - 5))));
-}
-__host__ __device__ constexpr float crumb_scale(int p) {
-  return p <= 4 ? (float)(1 << (2 * p)) : (float)(1 << (2 * (p - 5)));
-}
-// In-place INT4 code pair at nibble n (0..3) of both 16-bit halves:
-// c * 16^(n & 1) * 2^-24 each (nibbles 2, 3 come from x >> 8).
-__device__ __forceinline__ uint32_t nib_at(uint32_t x, uint32_t x8, int n) {
-  return (n < 2 ? x : x8) & ((n & 1) ? 0x00F000F0u : 0x000F000Fu);
-}
-
-// Copies of one stage: rows [0, nv) of the stage starting at the lane's
-// source pointers (already advanced to the stage's first row).
-template <int E, bool FULL>
-__device__ __forceinline__ void tc_issue(unsigned char* st, const unsigned char* gk,
-                                         const unsigned char* gv, const unsigned char* gks,
-                                         const unsigned char* gvs, int nv, int lane) {
-  using G = TG<E>;
-  if constexpr (E == 0) {
-    // 16 units per 256-byte row; the lane covers rows r, r + 2, ... at column c
-    const int r = lane >> 4, c = (lane & 15) * 16;
-    unsigned char* dk = st + G::KOFF + r * G::KROW + c;
-    unsigned char* dv = st + G::VOFF + r * G::KROW + c;
-#pragma unroll
-    for (int i = 0; i < G::TOK / 2; ++i)
-      if (FULL || 2 * i + r < nv) {
-        cp_async16(dk + i * 2 * G::KROW, gk + i * 2 * G::CROW);
-        cp_async16(dv + i * 2 * G::KROW, gv + i * 2 * G::CROW);
-      }
-  } else {
-    // codes: one contiguous block per array, unit lane + 32 i
-#pragma unroll
-    for (int i = 0; i < G::TOK * G::CU / 32; ++i)
-      if (FULL || (lane + 32 * i) / G::CU < nv) {
-        cp_async16(st + G::KOFF + lane * 16 + i * 512, gk + i * 512);
-        cp_async16(st + G::VOFF + lane * 16 + i * 512, gv + i * 512);
-      }
-    // scales: one 16-byte row per token, row lane
-    if (FULL || lane < nv) {
-      cp_async16(st + G::KSOFF + lane * 16, gks);
-      cp_async16(st + G::VSOFF + lane * 16, gvs);
-    }
-  }
-  cp_async_commit();
-}
 
 // Running state of the item in progress (one query head).
 struct TcState {
@@ -213,6 +141,7 @@ __device__ __forceinline__ void tc_query(TcQuery& Q, const __half* __restrict__ 
 }
 
 // One stage: scores of its subtiles, online softmax, B', values.
+// FULL: a stage of TOK valid rows (no row checks); otherwise rows [0, nv).
 template <int E, bool FULL>
 __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const unsigned char* st,
                                          int nv, int lane) {
@@ -241,8 +170,9 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
     } else {
       const unsigned char* kr = st + G::KOFF + (16 * u + gid) * G::CROW;
       if constexpr (E == 1) {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(kr + 16 * tig);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 8 * G::CROW + 16 * tig);
+        const int un = 16 * int4_unit(gid, tig);  // rows gid, gid + 8 share the swizzle
+        const uint4 w0 = *reinterpret_cast<const uint4*>(kr + un);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(kr + 8 * G::CROW + un);
         const uint32_t r0[4] = {w0.x, w0.y, w0.z, w0.w}, r1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -400,7 +330,8 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
       uint2 v[4];
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj)
-        v[jj] = *reinterpret_cast<const uint2*>(st + G::VOFF + (16 * u + tig + 4 * jj) * 64 + 8 * gid);
+        v[jj] = *reinterpret_cast<const uint2*>(st + G::VOFF + (16 * u + tig + 4 * jj) * 64 +
+                                                16 * int4_unit(tig + 4 * jj, gid >> 1) + 8 * (gid & 1));
       // halves of token pairs (0, 1) and (2, 3): dims 0-3, 4-7 (word a), 8-11, 12-15 (word b)
       la01[u] = __byte_perm(v[0].x, v[1].x, 0x5410); ha01[u] = __byte_perm(v[0].x, v[1].x, 0x7632);
       lb01[u] = __byte_perm(v[0].y, v[1].y, 0x5410); hb01[u] = __byte_perm(v[0].y, v[1].y, 0x7632);
@@ -485,74 +416,41 @@ __device__ __forceinline__ void tc_record(const TcState& S, int lane, int64_t w,
 // One run: tokens [T0, T1) of one region (the region's items j0, j0 + 1, ...
 // of IT tokens each; records w0, w0 + Hkv, ...), streamed through the ring.
 template <int E>
-__device__ __forceinline__ void tc_run(const unsigned char* __restrict__ regk,
-                                       const unsigned char* __restrict__ regv, uint64_t soff,
-                                       int T0, int T1, int IT, int64_t w0, int Hkv,
-                                       const __half* __restrict__ qh, float scale_log2,
-                                       unsigned char* ring, float* __restrict__ ws_acc,
-                                       float2* __restrict__ ws_ml) {
+__device__ __forceinline__ void tc_run(const TcRun& R, int Hkv, const __half* __restrict__ q,
+                                       float scale_log2, unsigned char* ring,
+                                       float* __restrict__ ws_acc, float2* __restrict__ ws_ml) {
   using G = TG<E>;
   const int lane = threadIdx.x & 31;
-  const int ntok = T1 - T0;
-  const int nst = (ntok + G::TOK - 1) / G::TOK;
-
-  // the lane's copy sources at the run's first stage; each stage advances them
-  const unsigned char *gk, *gv, *gks = nullptr, *gvs = nullptr;
-  if constexpr (E == 0) {
-    const int64_t row = (int64_t)T0 + (lane >> 4);
-    gk = regk + row * G::CROW + (lane & 15) * 16;
-    gv = regv + row * G::CROW + (lane & 15) * 16;
-  } else {
-    gk = regk + (int64_t)T0 * G::CROW + lane * 16;
-    gv = regv + (int64_t)T0 * G::CROW + lane * 16;
-    gks = regk + soff + ((int64_t)T0 + lane) * 16;
-    gvs = regv + soff + ((int64_t)T0 + lane) * 16;
-  }
-  constexpr int CSTEP = G::TOK * G::CROW, SSTEP = G::TOK * 16;
-  int issued = 0;
-  auto issue_next = [&]() {
-    if (issued < nst) {
-      unsigned char* st = ring + (issued % G::STAGES) * G::STAGE;
-      const int nv = min(G::TOK, ntok - issued * G::TOK);
-      if (nv == G::TOK)
-        tc_issue<E, true>(st, gk, gv, gks, gvs, nv, lane);
-      else
-        tc_issue<E, false>(st, gk, gv, gks, gvs, nv, lane);
-      gk += CSTEP;
-      gv += CSTEP;
-      if constexpr (E != 0) {
-        gks += SSTEP;
-        gvs += SSTEP;
-      }
-    } else {
-      cp_async_commit();
-    }
-    ++issued;
-  };
+  TcStream<E> cs;
+  cs.init(R.regk, R.regv, R.soff, R.T0, R.T1, lane);
 #pragma unroll 1
-  for (int s = 0; s < G::STAGES - 1; ++s) issue_next();
+  for (int s = 0; s < G::STAGES - 1; ++s) cs.issue_next(ring, lane);
 
   TcQuery Q;
-  tc_query<E>(Q, qh, scale_log2, lane);
+  tc_query<E>(Q, q + ((int64_t)R.b * Hkv + R.g) * 128, scale_log2, lane);
   TcState S;
   tc_reset(S);
-  int64_t w = w0;
+  int64_t w = R.w0;
+  const int item_stages = R.IT / G::TOK;  // item boundaries fall on stage boundaries
+  int left = item_stages, slot = 0;
 
 #pragma unroll 1
-  for (int k = 0; k < nst; ++k) {
-    issue_next();
+  for (int k = 0; k < cs.nst; ++k) {
+    cs.issue_next(ring, lane);
     cp_async_wait<G::STAGES - 1>();
     __syncwarp();
-    const unsigned char* st = ring + (k % G::STAGES) * G::STAGE;
-    const int nv = min(G::TOK, ntok - k * G::TOK);
+    const unsigned char* st = ring + slot * G::STAGE;
+    slot = slot + 1 == G::STAGES ? 0 : slot + 1;
+    const int nv = min(G::TOK, cs.ntok - k * G::TOK);
     if (nv == G::TOK)
       tc_stage<E, true>(S, Q, st, nv, lane);
     else
       tc_stage<E, false>(S, Q, st, nv, lane);
-    if (((k + 1) * G::TOK) % IT == 0 || k == nst - 1) {
+    if (--left == 0 || k == cs.nst - 1) {
       tc_record<E>(S, lane, w, ws_acc, ws_ml);
       tc_reset(S);
       w += Hkv;
+      left = item_stages;
     }
     __syncwarp();  // the stage is read before it is refilled
   }
@@ -564,69 +462,20 @@ __global__ void __launch_bounds__(32, kTcCtasPerSm)
 decode_mha_kernel(const unsigned char* __restrict__ layout, const unsigned char* __restrict__ packed,
                   const __half* __restrict__ q, float scale_log2, float* __restrict__ ws_acc,
                   float2* __restrict__ ws_ml, unsigned int* __restrict__ counter,
-                  int64_t capacity_items, unsigned int* status) {
+                  const int* __restrict__ tab, int B, int64_t capacity_items, unsigned int* status) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
-  if (h->magic != MQ_LAYOUT_MAGIC || h->head_dim != 128) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_BAD_LAYOUT);
-    return;
-  }
-  const int B = h->num_seqs, Hkv = h->num_kv_heads;
-  const int64_t total = (int64_t)h->total_items * Hkv;
-  if (total > capacity_items) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, MQ_DEV_WORKSPACE_TOO_SMALL);
-    return;
-  }
+  if (!tc_layout_ok(layout, B, capacity_items, status)) return;
+  const int Hkv = reinterpret_cast<const mq_layout_header*>(layout)->num_kv_heads;
   const int lane = threadIdx.x & 31;
-  const int64_t workers = (int64_t)gridDim.x;
-  // Items in region order: v = Hkv * item_begin[s] + g * item_count[s] + j for
-  // item j of segment s, kv-head g of a sequence (its record is
-  // (item_begin[s] + j) * Hkv + g).
-  for (;;) {
-    // guided claim: a group of up to kTcMaxGroup items, about the remaining
-    // work over twice the workers
-    unsigned int v0 = 0, cnt = 0;
-    if (lane == 0) {
-      const int64_t cur = (int64_t)*reinterpret_cast<volatile unsigned int*>(counter);
-      const int64_t want = (total - cur) / (2 * workers);
-      cnt = (unsigned int)(want < 1 ? 1 : (want > kTcMaxGroup ? kTcMaxGroup : want));
-      v0 = atomicAdd(counter, cnt);
-    }
-    v0 = __shfl_sync(0xffffffffu, v0, 0);
-    cnt = __shfl_sync(0xffffffffu, cnt, 0);
-    if ((int64_t)v0 >= total) break;
-    const int64_t v1 = min((int64_t)v0 + cnt, total);
-    for (int64_t v = v0; v < v1;) {
-      const int b = find_item_seq(layout, B, v / Hkv);
-      const mq_seq_layout* r = reinterpret_cast<const mq_seq_layout*>(layout + layout_seq_offset(b));
-      const int s = v < (int64_t)Hkv * r->item_begin[1] ? 0 : (v < (int64_t)Hkv * r->item_begin[2] ? 1 : 2);
-      const int64_t base = (int64_t)Hkv * r->item_begin[s];
-      const int cntr = r->item_count[s];
-      const int64_t u = v - base;
-      const int g = cntr > 0 ? (int)(u / cntr) : 0;
-      const int j = cntr > 0 ? (int)(u - (int64_t)g * cntr) : 0;
-      const int64_t vend = min(v1, base + (int64_t)(g + 1) * cntr);  // end of this region's items
-      const int IT = h->item_tokens[s];
-      const int T0 = j * IT;
-      const int T1 = (int)min((int64_t)r->seg_tokens[s], (int64_t)(j + (vend - v)) * IT);
-      if (cntr <= 0 || g >= Hkv || T1 <= T0) {
-        if (lane == 0) set_status(status, MQ_DEV_INDEX_RANGE);
-        break;
-      }
-      const unsigned char* regk = packed + r->seg_base[s] + (uint64_t)g * r->region_bytes[s];
-      const unsigned char* regv = regk + (uint64_t)Hkv * r->region_bytes[s];
-      const int64_t w0 = ((int64_t)r->item_begin[s] + j) * Hkv + g;
-      const __half* qh = q + ((int64_t)b * Hkv + g) * 128;
-      if (s == 0)
-        tc_run<0>(regk, regv, 0, T0, T1, IT, w0, Hkv, qh, scale_log2, smem_raw, ws_acc, ws_ml);
-      else if (s == 1)
-        tc_run<1>(regk, regv, r->scale_offset[1], T0, T1, IT, w0, Hkv, qh, scale_log2, smem_raw,
-                  ws_acc, ws_ml);
-      else
-        tc_run<2>(regk, regv, r->scale_offset[2], T0, T1, IT, w0, Hkv, qh, scale_log2, smem_raw,
-                  ws_acc, ws_ml);
-      v = vend;
-    }
+  TcRun R;
+  TcClaim C;
+  while (tc_next_run(R, C, layout, packed, tab, counter, status, lane)) {
+    if (R.s == 0)
+      tc_run<0>(R, Hkv, q, scale_log2, smem_raw, ws_acc, ws_ml);
+    else if (R.s == 1)
+      tc_run<1>(R, Hkv, q, scale_log2, smem_raw, ws_acc, ws_ml);
+    else
+      tc_run<2>(R, Hkv, q, scale_log2, smem_raw, ws_acc, ws_ml);
   }
 }
 
@@ -634,8 +483,8 @@ decode_mha_kernel(const unsigned char* __restrict__ layout, const unsigned char*
 
 cudaError_t launch_decode_mha(int64_t capacity_items, const unsigned char* layout,
                               const unsigned char* packed, const __half* q, float scale_log2,
-                              float* ws_acc, float2* ws_ml, unsigned int* counter,
-                              unsigned int* status, cudaStream_t stream) {
+                              float* ws_acc, float2* ws_ml, unsigned int* counter, int* tab,
+                              int B, int Hq, unsigned int* status, cudaStream_t stream) {
   cudaError_t e;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -650,9 +499,11 @@ cudaError_t launch_decode_mha(int64_t capacity_items, const unsigned char* layou
   int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
   if (grid > capacity_items) grid = capacity_items;
   if (grid <= 0) return cudaSuccess;
-  if ((e = cudaMemsetAsync(counter, 0, sizeof(unsigned int), stream)) != cudaSuccess) return e;
+  // the work order's prefix table, and the counter zeroed
+  tc_prep_kernel<<<1, 256, 0, stream>>>(layout, B, B * Hq, tab, counter);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   decode_mha_kernel<<<(unsigned)grid, 32, smem, stream>>>(layout, packed, q, scale_log2, ws_acc, ws_ml,
-                                                          counter, capacity_items, status);
+                                                          counter, tab, B, capacity_items, status);
   return cudaGetLastError();
 }
 

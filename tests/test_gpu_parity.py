@@ -38,6 +38,10 @@ CASES = {
     # kernel of that case (16-token stages: tails of 1, 15, 16, 17 tokens)
     "mha_f16_d128": Case(np.array([0, 1, 15, 16, 17, 127, 129, 1000, 3000], np.int32), 4, 4, 128,
                          32, "f16"),
+    # four query heads per kv-head, fp16 queries, d = 128: the grouped-query
+    # tensor-core kernel (tails of 1 to 33 tokens around its 16/32-token stages)
+    "gqa4_f16_tails": Case(np.array([1, 15, 16, 17, 31, 32, 33, 700, 0], np.int32), 8, 2, 128, 32,
+                           "f16"),
 }
 
 MAPS = {"mixed": (0.2, 0.5, 0.3), "fp16": (1, 0, 0), "int4": (0, 1, 0), "int2": (0, 0, 1)}
@@ -52,7 +56,8 @@ def _map(case, mix, seed=0):
 def test_layout_pack_decode_parity(name, mapname):
     case = CASES[name]
     if mapname != "mixed" and name not in ("ragged_gqa4", "tiny_like_f32", "gqa8_d128", "gqa4_d64",
-                                           "gqa4_f32_d64", "gqa8_f32_d128", "mha_f16_d128"):
+                                           "gqa4_f32_d64", "gqa8_f32_d128", "mha_f16_d128",
+                                           "gqa4_f16_tails"):
         pytest.skip("single-precision maps run on two cases")
     cmap = _map(case, MAPS[mapname], seed=zlib.crc32(name.encode()) & 0xFFFF)
     K, V, q = random_kv(case, seed=len(name))
