@@ -538,6 +538,7 @@ decode_combine_kernel(const unsigned char* __restrict__ layout, int Hq,
   __shared__ float s_m[NW], s_l[NW];
   __shared__ int s_last;
   const int S = gridDim.y, k = blockIdx.y;
+  pdl_wait();  // the partial records of the decode kernel
   const mq_layout_header* h = reinterpret_cast<const mq_layout_header*>(layout);
   const int Hkv = h->num_kv_heads;
   const int64_t bh = blockIdx.x;
@@ -1240,12 +1241,13 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
   const int64_t avg = max_items / Hq * QPG / (num_seqs > 0 ? num_seqs : 1);  // items per (b, h)
   const int S = (int)(avg / 64 < 1 ? 1 : (avg / 64 > kSplitMax ? kSplitMax : avg / 64));
   const dim3 grid((unsigned)heads, (unsigned)S);
-  if (partial)
-    decode_combine_kernel<D, QPG, true, 8><<<grid, 256, 0, stream>>>(layout, Hq, ws_acc, ws_ml, out,
-                                                                     split, done);
-  else
-    decode_combine_kernel<D, QPG, false, 8><<<grid, 256, 0, stream>>>(layout, Hq, ws_acc, ws_ml, out,
-                                                                      split, done);
+  const float* acc_c = ws_acc;
+  const float2* ml_c = ws_ml;
+  cudaError_t e2 = partial ? launch_pdl(decode_combine_kernel<D, QPG, true, 8>, grid, dim3(256), 0,
+                                        stream, layout, Hq, acc_c, ml_c, out, split, done)
+                           : launch_pdl(decode_combine_kernel<D, QPG, false, 8>, grid, dim3(256), 0,
+                                        stream, layout, Hq, acc_c, ml_c, out, split, done);
+  if (e2 != cudaSuccess) return e2;
   return cudaGetLastError();
 }
 

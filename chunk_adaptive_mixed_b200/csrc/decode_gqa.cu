@@ -143,9 +143,9 @@ __device__ __forceinline__ void gq_query(GqQuery& Q, const __half* __restrict__ 
 
 // Subtile u0 (tokens 16 u0 .. 16 u0 + 15) of a stage: scores of head tig,
 // online softmax, B', values.
-template <int E>
+template <int E, int u0, bool FULL>
 __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsigned char* st,
-                                       int u0, int nv, int lane) {
+                                       int nv, int lane) {
   using G = TG<E>;
   constexpr int SUB = 1;
   const int gid = lane >> 2, tig = lane & 3;
@@ -223,8 +223,8 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
       v1 = fmaf(d1, Q.sfac, m1);
     }
     // rows past the item's end hold stale bytes (maybe not numbers): select
-    x[u][0] = (16 * (u0 + u) + gid < nv) ? v0 : -INFINITY;
-    x[u][1] = (16 * (u0 + u) + gid + 8 < nv) ? v1 : -INFINITY;
+    x[u][0] = (FULL || 16 * (u0 + u) + gid < nv) ? v0 : -INFINITY;
+    x[u][1] = (FULL || 16 * (u0 + u) + gid + 8 < nv) ? v1 : -INFINITY;
   }
 
   // ---- online softmax of head tig, reference moved lazily
@@ -273,7 +273,7 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
     const uint32_t l23 = h2_bits(__floats2half2_rn(P[0][2] - f23.x, P[0][3] - f23.y));
     const uint32_t bb0 = hl ? l01 : h01, bb1 = hl ? l23 : h23;
     unsigned char* stw = const_cast<unsigned char*>(st);
-    if (nv < 16) {  // stale rows may not be numbers, and 0 * NaN is NaN
+    if (!FULL && nv < 16) {  // stale rows may not be numbers, and 0 * NaN is NaN
       constexpr int RU = 256 / 16;
       for (int i = lane; i < (16 - nv) * RU; i += 32)
         *reinterpret_cast<uint4*>(stw + G::VOFF + (nv + i / RU) * G::KROW + (i % RU) * 16) =
@@ -301,7 +301,7 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
       for (int j = 0; j < 4; ++j) {
         const int row = 16 * (u0 + u) + tig + 4 * j;
         uint2 raw = *reinterpret_cast<const uint2*>(st + G::VSOFF + row * 16 + 4 * ga);
-        if (row >= nv) raw = make_uint2(0u, 0u);  // stale scales may not be numbers
+        if (!FULL && row >= nv) raw = make_uint2(0u, 0u);  // stale scales may not be numbers
         const float2 a = half2_bits_to_float2(raw.x), b = half2_bits_to_float2(raw.y);
         vs[j][0] = a.x; vm[j][0] = a.y;
         vs[j][1] = b.x; vm[j][1] = b.y;
@@ -404,15 +404,18 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
   }
 }
 
-// One stage: its subtiles one after another (one copy of the subtile code,
-// which keeps the kernel's instruction footprint small).
+// One stage: its subtiles one after another; a full stage (TOK rows) needs
+// no row checks, a tail stage skips an empty second subtile.
 template <int E>
 __device__ __forceinline__ void gq_stage(GqState& S, const GqQuery& Q, const unsigned char* st,
                                          int nv, int lane) {
-#pragma unroll 1
-  for (int u0 = 0; u0 < TG<E>::SUB; ++u0) {
-    if (16 * u0 >= nv) break;  // empty subtile of a tail stage
-    gq_sub<E>(S, Q, st, u0, nv, lane);
+  if (nv == TG<E>::TOK) {
+    gq_sub<E, 0, true>(S, Q, st, nv, lane);
+    if constexpr (TG<E>::SUB == 2) gq_sub<E, 1, true>(S, Q, st, nv, lane);
+  } else {
+    gq_sub<E, 0, false>(S, Q, st, nv, lane);
+    if constexpr (TG<E>::SUB == 2)
+      if (nv > 16) gq_sub<E, 1, false>(S, Q, st, nv, lane);
   }
 }
 
@@ -498,6 +501,8 @@ decode_gqa_kernel(const unsigned char* __restrict__ layout, const unsigned char*
                   float2* __restrict__ ws_ml, unsigned int* __restrict__ counter,
                   const int* __restrict__ tab, int B, int64_t capacity_items, unsigned int* status) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
+  pdl_wait();     // the prep kernel's table and counters
+  pdl_trigger();  // the combine may launch; it waits for this kernel
   if (!tc_layout_ok(layout, B, capacity_items, status)) return;
   const int Hkv = reinterpret_cast<const mq_layout_header*>(layout)->num_kv_heads;
   const int lane = threadIdx.x & 31;
@@ -536,9 +541,8 @@ cudaError_t launch_decode_gqa4(int64_t capacity_items, const unsigned char* layo
   // the work order's prefix table, and the counter zeroed
   tc_prep_kernel<<<1, 256, 0, stream>>>(layout, B, B * Hq, tab, counter);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_gqa_kernel<<<(unsigned)grid, 32, smem, stream>>>(layout, packed, q, scale_log2, ws_acc, ws_ml,
-                                                          counter, tab, B, capacity_items, status);
-  return cudaGetLastError();
+  return launch_pdl(decode_gqa_kernel, dim3((unsigned)grid), dim3(32), smem, stream, layout, packed, q,
+                    scale_log2, ws_acc, ws_ml, counter, tab, B, capacity_items, status);
 }
 
 }  // namespace mqkv

@@ -464,6 +464,8 @@ decode_mha_kernel(const unsigned char* __restrict__ layout, const unsigned char*
                   float2* __restrict__ ws_ml, unsigned int* __restrict__ counter,
                   const int* __restrict__ tab, int B, int64_t capacity_items, unsigned int* status) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
+  pdl_wait();     // the prep kernel's table and counters
+  pdl_trigger();  // the combine may launch; it waits for this kernel
   if (!tc_layout_ok(layout, B, capacity_items, status)) return;
   const int Hkv = reinterpret_cast<const mq_layout_header*>(layout)->num_kv_heads;
   const int lane = threadIdx.x & 31;
@@ -502,9 +504,8 @@ cudaError_t launch_decode_mha(int64_t capacity_items, const unsigned char* layou
   // the work order's prefix table, and the counter zeroed
   tc_prep_kernel<<<1, 256, 0, stream>>>(layout, B, B * Hq, tab, counter);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_mha_kernel<<<(unsigned)grid, 32, smem, stream>>>(layout, packed, q, scale_log2, ws_acc, ws_ml,
-                                                          counter, tab, B, capacity_items, status);
-  return cudaGetLastError();
+  return launch_pdl(decode_mha_kernel, dim3((unsigned)grid), dim3(32), smem, stream, layout, packed, q,
+                    scale_log2, ws_acc, ws_ml, counter, tab, B, capacity_items, status);
 }
 
 }  // namespace mqkv

@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(256)
 tc_prep_kernel(const unsigned char* __restrict__ layout, int B, int nheads, int* __restrict__ tab,
                unsigned int* __restrict__ counter) {
   __shared__ int red[33];
+  pdl_trigger();  // the decode kernel may launch now; it waits for this one
   for (int i = threadIdx.x; i <= nheads; i += blockDim.x) counter[i] = 0u;
   for (int s = 0; s < kNumExperts; ++s) {
     int carry = 0;
