@@ -23,12 +23,16 @@
 // Values: O^T[128 dims x 8 columns] += Vhat^T . B'_g per m-tile, where m-tile
 //   mt covers dims 16 mt .. 16 mt + 15 (group g = mt / 2) and column
 //   (h, hl) of B'_g holds p_th * s_tg split into fp16 high (hl = 0) and low
-//   (hl = 1) parts.  Lane (gid, tig) accumulates head tig for dims
-//   16 mt + gid and 16 mt + gid + 8.  The code pair of one dim and two tokens
-//   is one byte permute and one mask; its power-of-two position factor
-//   depends only on gid and is removed from the finished accumulator.
-//   Partner lanes (columns hl = 0, 1 of a head) each form both parts for two
-//   of the four groups and exchange the halves the other needs.
+//   (hl = 1) parts.  Lane (gid, tig) accumulates head tig for rows gid and
+//   gid + 8 of every m-tile.  INT2: the rows are dims 16 mt + gid (+8), the
+//   code pair of one dim and two tokens is one byte permute and one mask.
+//   INT4: a group is one 16-byte unit of a token row, so a transposed
+//   ldmatrix puts a dim's codes of two tokens side by side; m-tile
+//   2 g + sh holds group g's dims 4 i + 2 sh (rows i) and 4 i + 2 sh + 1
+//   (rows i + 8).  The codes' power-of-two position factors are removed
+//   from the finished accumulator.  Partner lanes (columns hl = 0, 1 of a
+//   head) each form both parts for two of the four groups and exchange the
+//   halves the other needs.
 #include "decode_tc.cuh"
 
 namespace mqkv {
@@ -36,9 +40,15 @@ namespace {
 
 constexpr int kG = 4;  // query heads per kv-head
 
+// Token of B' row pair slot j (0..3) on a lane with index tig in its quad.
+template <int E>
+__device__ __forceinline__ int gq_tau(int tig, int j) {
+  return E == 2 ? tig + 4 * j : 2 * tig + (j & 1) + 8 * (j >> 1);
+}
+
 // Running state of the item in progress.
 struct GqState {
-  float o[8][4];   // O^T tiles: head tig, dims 16 mt + gid (+8), columns hi / lo
+  float o[8][4];   // O^T tiles: head tig, rows gid, gid + 8 of m-tile mt, columns hi / lo
   float m, m8, l;  // head tig: reference, reference + 8, sum over this lane's rows
   uint64_t bias2;  // head gid / 2, groups 2 (gid & 1) + {0, 1}: sum over this lane's tokens of p * min
   float down, vlim;
@@ -252,15 +262,15 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
     p[u][1] = ex2_ftz(x[u][1] - S.m);
     S.l += p[u][0] + p[u][1];
   }
-  // this lane's B' rows are tokens tau_j (INT: tig + 4 j, the V operand's
-  // token pairs; FP16: the ldmatrix order 2 tig + (j & 1) + 8 (j >> 1)) of
-  // head gid / 2
+  // this lane's B' rows are tokens tau_j of head gid / 2: the V operand's
+  // token pairs, tig + 4 j for INT2, the transposed-ldmatrix order
+  // 2 tig + (j & 1) + 8 (j >> 1) otherwise
   float P[SUB][4];
 #pragma unroll
   for (int u = 0; u < SUB; ++u)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int tau = E == 0 ? 2 * tig + (j & 1) + 8 * (j >> 1) : tig + 4 * j;
+      const int tau = gq_tau<E>(tig, j);
       P[u][j] = __shfl_sync(0xffffffffu, p[u][tau >> 3], 4 * (tau & 7) + (gid >> 1));
     }
 
@@ -299,7 +309,7 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
       float vs[4][2], vm[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int row = 16 * (u0 + u) + tig + 4 * j;
+        const int row = 16 * (u0 + u) + gq_tau<E>(tig, j);
         uint2 raw = *reinterpret_cast<const uint2*>(st + G::VSOFF + row * 16 + 4 * ga);
         if (!FULL && row >= nv) raw = make_uint2(0u, 0u);  // stale scales may not be numbers
         const float2 a = half2_bits_to_float2(raw.x), b = half2_bits_to_float2(raw.y);
@@ -351,10 +361,10 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
           bb[2 + k][1] = hl ? own1 : rcv1;
         }
       }
-      // A operand: m-tile mt covers dims 16 mt .. 16 mt + 15 (group mt / 2);
-      // row gid (gid + 8) is dim 16 mt + gid (+ 8): one byte of each of two
-      // token rows, put side by side by a byte permute, then one mask
+      // A operand: m-tile mt covers 16 dims of group mt / 2
       if constexpr (E == 2) {
+        // row gid (gid + 8) is dim 16 mt + gid (+ 8): one byte of each of two
+        // token rows, put side by side by a byte permute, then one mask
         // word mt of a row: rows 0-7 in its low half (byte gid / 4), 8-15 in its high half
         const uint32_t kA = gid >> 2, kB = 2 + (gid >> 2);
         const uint32_t selA = kA | (kA << 4) | ((kA + 4) << 8) | ((kA + 4) << 12);
@@ -365,7 +375,8 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
           uint4 w[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            w[j] = *reinterpret_cast<const uint4*>(st + G::VOFF + (16 * (u0 + u) + tig + 4 * j) * 32 + 16 * hv);
+            w[j] = *reinterpret_cast<const uint4*>(st + G::VOFF + (16 * (u0 + u) + tig + 4 * j) * 32 +
+                                                   16 * int2_unit(tig + 4 * j, hv));
           const uint32_t w0[4] = {w[0].x, w[0].y, w[0].z, w[0].w}, w1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
           const uint32_t w2[4] = {w[2].x, w[2].y, w[2].z, w[2].w}, w3[4] = {w[3].x, w[3].y, w[3].z, w[3].w};
 #pragma unroll
@@ -377,26 +388,26 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
           }
         }
       } else {
-        // words 2 mt (rows 0-7) and 2 mt + 1 (rows 8-15): nibble gid, byte gid / 2
-        const uint32_t kk = gid >> 1;
-        const uint32_t sel = kk | (kk << 4) | ((kk + 4) << 8) | ((kk + 4) << 12);
-        const uint32_t M = 0x000F000Fu << (4 * (gid & 1));
+        // a transposed ldmatrix of 8 token rows x one 16-byte unit (one group)
+        // gives lane (gid, tig) 16-bit word gid (dims 4 gid .. 4 gid + 3 of
+        // the group) of tokens 2 tig (low half) and 2 tig + 1 (high half):
+        // m-tile 2 g + sh takes nibbles 2 sh (rows gid) and 2 sh + 1 (rows
+        // gid + 8) of group g, two masks per pair of tokens
+        const int j = lane >> 3;
+        const int row = 16 * (u0 + u) + (lane & 7) + 8 * (j & 1);
+        const uint32_t vrow = smem_addr(st + G::VOFF) + row * 64;
 #pragma unroll
-        for (int qv = 0; qv < 4; ++qv) {
-          uint4 w[4];
+        for (int hv = 0; hv < 2; ++hv) {
+          uint32_t r[4];  // (group 2 hv, tokens 0-7), (2 hv, 8-15), (2 hv + 1, 0-7), (2 hv + 1, 8-15)
+          ldsm_x4_t(r, vrow + 16 * int4_unit(row, 2 * hv + (j >> 1)));
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            w[j] = *reinterpret_cast<const uint4*>(st + G::VOFF + (16 * (u0 + u) + tig + 4 * j) * 64 +
-                                                   16 * int4_unit(tig + 4 * j, qv));
-          const uint32_t w0[4] = {w[0].x, w[0].y, w[0].z, w[0].w}, w1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
-          const uint32_t w2[4] = {w[2].x, w[2].y, w[2].z, w[2].w}, w3[4] = {w[3].x, w[3].y, w[3].z, w[3].w};
-#pragma unroll
-          for (int mm = 0; mm < 2; ++mm) {
-            const int mt = 2 * qv + mm;
-            mma16816(S.o[mt], __byte_perm(w0[2 * mm], w1[2 * mm], sel) & M,
-                     __byte_perm(w0[2 * mm + 1], w1[2 * mm + 1], sel) & M,
-                     __byte_perm(w2[2 * mm], w3[2 * mm], sel) & M,
-                     __byte_perm(w2[2 * mm + 1], w3[2 * mm + 1], sel) & M, bb[mt / 2][0], bb[mt / 2][1]);
+          for (int gg = 0; gg < 2; ++gg) {
+            const int g = 2 * hv + gg;
+            const uint32_t lo = r[2 * gg], hi = r[2 * gg + 1], lo8 = lo >> 8, hi8 = hi >> 8;
+            mma16816(S.o[2 * g], lo & 0x000F000Fu, lo & 0x00F000F0u, hi & 0x000F000Fu, hi & 0x00F000F0u,
+                     bb[g][0], bb[g][1]);
+            mma16816(S.o[2 * g + 1], lo8 & 0x000F000Fu, lo8 & 0x00F000F0u, hi8 & 0x000F000Fu,
+                     hi8 & 0x00F000F0u, bb[g][0], bb[g][1]);
           }
         }
       }
@@ -442,15 +453,28 @@ __device__ __forceinline__ void gq_record(const GqState& S, int lane, int64_t w,
     bias[1] = __shfl_sync(0xffffffffu, b1, 8 * tig);
     bias[2] = __shfl_sync(0xffffffffu, b0, 8 * tig + 4);
     bias[3] = __shfl_sync(0xffffffffu, b1, 8 * tig + 4);
-    // 2^A, the codes' 2^-24 and this lane's position factor
-    const float pos = E == 1 ? ((gid & 1) ? 16.f : 1.f) : (float)(1 << (2 * (gid & 3)));
+    // 2^A, the codes' 2^-24 and (INT2) this lane's position factor
+    const float pos = E == 1 ? 1.f : (float)(1 << (2 * (gid & 3)));
     f = 16777216.0f / S.down / pos;
   }
   float* dst = ws_acc + ((size_t)w * kG + tig) * 128;
+  if constexpr (E == 1) {
+    // m-tile 2 g + sh: rows gid, gid + 8 are dims 32 g + 4 gid + 2 sh and
+    // 32 g + 4 gid + 2 sh + 1 (nibbles at bit 4 carry a factor 16)
+    const float f16 = f * 0.0625f;
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    dst[16 * mt + gid] = fmaf(S.o[mt][0] + S.o[mt][1], f, bias[mt / 2]);
-    dst[16 * mt + gid + 8] = fmaf(S.o[mt][2] + S.o[mt][3], f, bias[mt / 2]);
+    for (int g = 0; g < 4; ++g)
+      *reinterpret_cast<float4*>(dst + 32 * g + 4 * gid) =
+          make_float4(fmaf(S.o[2 * g][0] + S.o[2 * g][1], f, bias[g]),
+                      fmaf(S.o[2 * g][2] + S.o[2 * g][3], f16, bias[g]),
+                      fmaf(S.o[2 * g + 1][0] + S.o[2 * g + 1][1], f, bias[g]),
+                      fmaf(S.o[2 * g + 1][2] + S.o[2 * g + 1][3], f16, bias[g]));
+  } else {
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      dst[16 * mt + gid] = fmaf(S.o[mt][0] + S.o[mt][1], f, bias[mt / 2]);
+      dst[16 * mt + gid + 8] = fmaf(S.o[mt][2] + S.o[mt][3], f, bias[mt / 2]);
+    }
   }
   if (gid == 0) ws_ml[(size_t)w * kG + tig] = make_float2(S.m, l);
 }

@@ -32,9 +32,10 @@
 // operand slot is divided out of the matching query element (scores; the
 // query is first brought to [2^14, 2^15) by one power of two so the divided
 // elements stay normal) or out of the finished accumulator (values).  For the
-// value product the A operand pairs two tokens of one dim: byte permutes
-// interleave the 16-bit halves of two token rows, then masks pick each dim's
-// code pair.
+// value product the A operand pairs two tokens of one dim: a transposed
+// ldmatrix over token rows puts the same 16-bit word of two tokens side by
+// side, then masks pick each dim's code pair (so an m-tile's rows are dims in
+// the order of their bit positions, undone when the record is written).
 //
 // Work: one warp per CTA (12 per SM) is a persistent worker.  Work items are
 // numbered region by region — (sequence, segment, kv-head), then the items of
@@ -233,8 +234,8 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
 #pragma unroll
       for (int i = 0; i < 4; ++i) S.o[mt][i] *= a;
   }
-  // this lane's B' rows are tokens tau_j of each subtile: INT tig + 4 j (the
-  // V operand's token pairs), FP16 the ldmatrix order 2 tig + (j & 1) + 8 (j >> 1)
+  // this lane's B' rows are tokens tau_j = 2 tig + (j & 1) + 8 (j >> 1) of
+  // each subtile, the token pairs of a transposed ldmatrix
   float P[SUB][4];
 #pragma unroll
   for (int u = 0; u < SUB; ++u) {
@@ -242,7 +243,7 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
     const float pv = (tig & 1) ? p1 : p0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int tau = E == 0 ? 2 * tig + (j & 1) + 8 * (j >> 1) : tig + 4 * j;
+      const int tau = 2 * tig + (j & 1) + 8 * (j >> 1);
       P[u][j] = __shfl_sync(0xffffffffu, pv, 4 * (tau & 7) + (tau >> 3));
     }
     S.l += (P[u][0] + P[u][1]) + (P[u][2] + P[u][3]);
@@ -264,7 +265,7 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
     for (int u = 0; u < SUB; ++u)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int row = 16 * u + tig + 4 * j;
+        const int row = 16 * u + 2 * tig + (j & 1) + 8 * (j >> 1);
         uint32_t raw = *reinterpret_cast<const uint32_t*>(st + G::VSOFF + row * 16 + 4 * g);
         if (!FULL) raw = row < nv ? raw : 0u;  // stale scales may not be numbers
         const float2 f = half2_bits_to_float2(raw);
@@ -323,49 +324,44 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
       ldsm_x4_t(a, arow + mt * 32);
       mma16816(S.o[mt], a[0], a[1], a[2], a[3], bb[0][0], bb[0][1]);
     }
-  } else if constexpr (E == 1) {
-    uint32_t la01[SUB], ha01[SUB], lb01[SUB], hb01[SUB], la23[SUB], ha23[SUB], lb23[SUB], hb23[SUB];
-#pragma unroll
-    for (int u = 0; u < SUB; ++u) {
-      uint2 v[4];
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        v[jj] = *reinterpret_cast<const uint2*>(st + G::VOFF + (16 * u + tig + 4 * jj) * 64 +
-                                                16 * int4_unit(tig + 4 * jj, gid >> 1) + 8 * (gid & 1));
-      // halves of token pairs (0, 1) and (2, 3): dims 0-3, 4-7 (word a), 8-11, 12-15 (word b)
-      la01[u] = __byte_perm(v[0].x, v[1].x, 0x5410); ha01[u] = __byte_perm(v[0].x, v[1].x, 0x7632);
-      lb01[u] = __byte_perm(v[0].y, v[1].y, 0x5410); hb01[u] = __byte_perm(v[0].y, v[1].y, 0x7632);
-      la23[u] = __byte_perm(v[2].x, v[3].x, 0x5410); ha23[u] = __byte_perm(v[2].x, v[3].x, 0x7632);
-      lb23[u] = __byte_perm(v[2].y, v[3].y, 0x5410); hb23[u] = __byte_perm(v[2].y, v[3].y, 0x7632);
-    }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-      for (int u = 0; u < SUB; ++u) {
-        const uint32_t xa01 = mt < 4 ? la01[u] : ha01[u], xb01 = mt < 4 ? lb01[u] : hb01[u];
-        const uint32_t xa23 = mt < 4 ? la23[u] : ha23[u], xb23 = mt < 4 ? lb23[u] : hb23[u];
-        const int nb = mt & 3;
-        mma16816(S.o[mt], nib_at(xa01, xa01 >> 8, nb), nib_at(xb01, xb01 >> 8, nb),
-                 nib_at(xa23, xa23 >> 8, nb), nib_at(xb23, xb23 >> 8, nb), bb[u][0], bb[u][1]);
-      }
   } else {
-    uint32_t l01[SUB], h01[SUB], l23[SUB], h23[SUB];
+    // a transposed ldmatrix of 8 token rows x one 16-byte unit gives lane
+    // (gid, tig) 16-bit word gid of the unit for tokens 2 tig (low half) and
+    // 2 tig + 1 (high half); masks then pick one dim's code pair
+    const int j = lane >> 3;
 #pragma unroll
     for (int u = 0; u < SUB; ++u) {
-      uint32_t v[4];
+      const int row = 16 * u + (lane & 7) + 8 * (j & 1);
+      if constexpr (E == 1) {
+        // unit = group; m-tile 2 g + sh takes nibbles 2 sh (rows gid) and
+        // 2 sh + 1 (rows gid + 8) of word gid: dims 32 g + 4 gid + 2 sh (+1)
+        const uint32_t vrow = smem_addr(st + G::VOFF) + row * 64;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        v[jj] = *reinterpret_cast<const uint32_t*>(st + G::VOFF + (16 * u + tig + 4 * jj) * 32 + 4 * gid);
-      l01[u] = __byte_perm(v[0], v[1], 0x5410); h01[u] = __byte_perm(v[0], v[1], 0x7632);
-      l23[u] = __byte_perm(v[2], v[3], 0x5410); h23[u] = __byte_perm(v[2], v[3], 0x7632);
+        for (int hv = 0; hv < 2; ++hv) {
+          uint32_t r[4];  // (group 2 hv, tokens 0-7), (2 hv, 8-15), (2 hv + 1, 0-7), (2 hv + 1, 8-15)
+          ldsm_x4_t(r, vrow + 16 * int4_unit(row, 2 * hv + (j >> 1)));
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            const int mt = 2 * (2 * hv + gg);
+            const uint32_t lo = r[2 * gg], hi = r[2 * gg + 1], lo8 = lo >> 8, hi8 = hi >> 8;
+            mma16816(S.o[mt], lo & 0x000F000Fu, lo & 0x00F000F0u, hi & 0x000F000Fu, hi & 0x00F000F0u,
+                     bb[u][0], bb[u][1]);
+            mma16816(S.o[mt + 1], lo8 & 0x000F000Fu, lo8 & 0x00F000F0u, hi8 & 0x000F000Fu,
+                     hi8 & 0x00F000F0u, bb[u][0], bb[u][1]);
+          }
+        }
+      } else {
+        // units 0, 1 hold dims 0-63, 64-127; m-tile p takes crumb p of word
+        // gid: rows gid, gid + 8 are dims 8 gid + p and 64 + 8 gid + p
+        uint32_t r[4];  // (unit 0, tokens 0-7), (0, 8-15), (1, 0-7), (1, 8-15)
+        ldsm_x4_t(r, smem_addr(st + G::VOFF) + row * 32 + 16 * int2_unit(row, j >> 1));
+        const uint32_t s0 = r[0] >> 10, s1 = r[1] >> 10, s2 = r[2] >> 10, s3 = r[3] >> 10;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+          mma16816(S.o[mt], crumb_at(r[0], s0, mt), crumb_at(r[2], s2, mt), crumb_at(r[1], s1, mt),
+                   crumb_at(r[3], s3, mt), bb[u][0], bb[u][1]);
+      }
     }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-      for (int u = 0; u < SUB; ++u)
-        mma16816(S.o[mt], crumb_at(l01[u], l01[u] >> 10, mt), crumb_at(h01[u], h01[u] >> 10, mt),
-                 crumb_at(l23[u], l23[u] >> 10, mt), crumb_at(h23[u], h23[u] >> 10, mt), bb[u][0],
-                 bb[u][1]);
   }
 }
 
@@ -389,25 +385,39 @@ __device__ __forceinline__ void tc_record(const TcState& S, int lane, int64_t w,
       }
     }
   } else {
-    float bias = lo2(S.bias2) + hi2(S.bias2);
+    float bias = lo2(S.bias2) + hi2(S.bias2);  // group gid / 2, this lane's tokens
     bias += __shfl_xor_sync(0xffffffffu, bias, 1);
     bias += __shfl_xor_sync(0xffffffffu, bias, 2);
-    // lanes whose columns (2 tig, 2 tig + 1) are their own dims' group hold
-    // dims 16 gid + mt (row gid) and 16 gid + 8 + mt (row gid + 8)
-    if (tig == (gid >> 1)) {
-      const float up = 16777216.0f / S.down;  // 2^A and the codes' 2^-24
-      float r0[8], r1[8];
+    // columns (2 tig, 2 tig + 1) are group tig's: a lane writes the dims of
+    // group tig among its rows, with that group's sum of p * min
+    bias = __shfl_sync(0xffffffffu, bias, 8 * tig);
+    const float up = 16777216.0f / S.down;  // 2^A and the codes' 2^-24
+    if constexpr (E == 1) {
+      // m-tiles 2 tig, 2 tig + 1: dims 32 tig + 4 gid + (0, 1, 2, 3), the odd
+      // ones from nibbles at bit 4 (factor 16)
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const float f = up / (E == 1 ? ((mt & 1) ? 16.f : 1.f) : crumb_scale(mt));
-        r0[mt] = fmaf(S.o[mt][0] + S.o[mt][1], f, bias);
-        r1[mt] = fmaf(S.o[mt][2] + S.o[mt][3], f, bias);
+      for (int g = 0; g < 4; ++g)
+        if (tig == g)
+          v = make_float4(S.o[2 * g][0] + S.o[2 * g][1], S.o[2 * g][2] + S.o[2 * g][3],
+                          S.o[2 * g + 1][0] + S.o[2 * g + 1][1], S.o[2 * g + 1][2] + S.o[2 * g + 1][3]);
+      *reinterpret_cast<float4*>(dst + 32 * tig + 4 * gid) =
+          make_float4(fmaf(v.x, up, bias), fmaf(v.y, up * 0.0625f, bias), fmaf(v.z, up, bias),
+                      fmaf(v.w, up * 0.0625f, bias));
+    } else {
+      // rows gid hold dims 8 gid + mt (group gid / 4), rows gid + 8 dims
+      // 64 + 8 gid + mt (group 2 + gid / 4)
+      const bool upper = tig >= 2;
+      if (tig == (gid >> 2) + (upper ? 2 : 0)) {
+        float r[8];
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+          r[mt] = fmaf(upper ? S.o[mt][2] + S.o[mt][3] : S.o[mt][0] + S.o[mt][1], up / crumb_scale(mt),
+                       bias);
+        float4* d4 = reinterpret_cast<float4*>(dst + (upper ? 64 : 0) + 8 * gid);
+        d4[0] = make_float4(r[0], r[1], r[2], r[3]);
+        d4[1] = make_float4(r[4], r[5], r[6], r[7]);
       }
-      float4* d4 = reinterpret_cast<float4*>(dst + 16 * gid);
-      d4[0] = make_float4(r0[0], r0[1], r0[2], r0[3]);
-      d4[1] = make_float4(r0[4], r0[5], r0[6], r0[7]);
-      d4[2] = make_float4(r1[0], r1[1], r1[2], r1[3]);
-      d4[3] = make_float4(r1[4], r1[5], r1[6], r1[7]);
     }
   }
   if (lane == 0) ws_ml[w] = make_float2(S.m, l);

@@ -62,6 +62,10 @@ __device__ __forceinline__ uint32_t nib_at(uint32_t x, uint32_t x8, int n) {
 // rows r and r + 2 fall on different banks.  (Row parity and rows 8 apart keep
 // the same pattern; unit r + 32 i shares row r's.)
 __device__ __forceinline__ int int4_unit(int row, int c) { return c ^ ((row >> 1) & 3); }
+// Staged INT2 value rows (32 bytes, two units) keep unit c of row r at unit
+// c ^ ((r >> 2) & 1), so that the eight rows of a transposed ldmatrix phase
+// fall on eight different 16-byte bank groups.  Key rows are not swizzled.
+__device__ __forceinline__ int int2_unit(int row, int c) { return c ^ ((row >> 2) & 1); }
 
 // Copies of one stage: rows [0, nv) of the stage starting at the lane's
 // source pointers (already advanced to the stage's first row).
@@ -83,13 +87,15 @@ __device__ __forceinline__ void tc_issue(unsigned char* st, const unsigned char*
       }
   } else {
     // codes: one contiguous block per array, unit lane + 32 i; INT4 rows keep
-    // their four units XOR-swizzled (int4_unit)
+    // their four units XOR-swizzled (int4_unit), INT2 value rows their two
+    // (int2_unit)
     const int dl = E == 1 ? (lane >> 2) * 64 + 16 * int4_unit(lane >> 2, lane & 3) : lane * 16;
+    const int dlv = E == 1 ? dl : (lane >> 1) * 32 + 16 * int2_unit(lane >> 1, lane & 1);
 #pragma unroll
     for (int i = 0; i < G::TOK * G::CU / 32; ++i)
       if (FULL || (lane + 32 * i) / G::CU < nv) {
         cp_async16(st + G::KOFF + dl + i * 512, gk + i * 512);
-        cp_async16(st + G::VOFF + dl + i * 512, gv + i * 512);
+        cp_async16(st + G::VOFF + dlv + i * 512, gv + i * 512);
       }
     // scales: one 16-byte row per token, row lane
     if (FULL || lane < nv) {
