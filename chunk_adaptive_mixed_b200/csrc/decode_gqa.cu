@@ -20,19 +20,23 @@
 //   one MMA per k-step.  Lane (gid, tig) then holds, for its tokens gid and
 //   gid + 8, the four groups' code dot products of head tig, applies each
 //   group's scale and min and has the score of head tig without any exchange.
-// Values: O^T[128 dims x 8 columns] += Vhat^T . B'_g per m-tile, where m-tile
-//   mt covers dims 16 mt .. 16 mt + 15 (group g = mt / 2) and column
-//   (h, hl) of B'_g holds p_th * s_tg split into fp16 high (hl = 0) and low
-//   (hl = 1) parts.  Lane (gid, tig) accumulates head tig for rows gid and
-//   gid + 8 of every m-tile.  INT2: the rows are dims 16 mt + gid (+8), the
-//   code pair of one dim and two tokens is one byte permute and one mask.
-//   INT4: a group is one 16-byte unit of a token row, so a transposed
-//   ldmatrix puts a dim's codes of two tokens side by side; m-tile
-//   2 g + sh holds group g's dims 4 i + 2 sh (rows i) and 4 i + 2 sh + 1
-//   (rows i + 8).  The codes' power-of-two position factors are removed
-//   from the finished accumulator.  Partner lanes (columns hl = 0, 1 of a
-//   head) each form both parts for two of the four groups and exchange the
-//   halves the other needs.
+// Values: O^T[128 dims x 8 columns] += Vhat^T . B' per m-tile, B' holding
+//   p_th * s_tg split into an fp16 high part and the fp16 remainder.  A
+//   transposed ldmatrix of token rows puts one 16-bit word of two tokens
+//   side by side, so a mask gives a dim's code pair.  Lane (gid, tig)
+//   accumulates head tig for rows gid and gid + 8 of every m-tile.
+//   INT4: a group is one 16-byte unit of a token row; m-tile 2 g + sh holds
+//   group g's dims 4 i + 2 sh (rows i) and 4 i + 2 sh + 1 (rows i + 8), and
+//   B'_g's column (h, hl) is head h's high (hl = 0) or low (hl = 1) part.
+//   Partner lanes (the two columns of a head) each form both parts for two
+//   of the four groups and exchange the halves the other needs.
+//   INT2: a 16-byte unit holds two groups; m-tile 4 k + p holds dims
+//   64 k + 8 i + p (rows i) and 64 k + 8 i + p + 4 (rows i + 8), both in
+//   group 2 k + i / 4, and B'_k's column (h, gp) is head h, group 2 k + gp:
+//   two MMAs per m-tile, high parts then low parts, into one accumulator,
+//   of whose columns a lane keeps the one of its rows' group.
+//   The codes' power-of-two position factors are removed from the finished
+//   accumulator.
 #include "decode_tc.cuh"
 
 namespace mqkv {
@@ -41,16 +45,14 @@ namespace {
 constexpr int kG = 4;  // query heads per kv-head
 
 // Token of B' row pair slot j (0..3) on a lane with index tig in its quad.
-template <int E>
-__device__ __forceinline__ int gq_tau(int tig, int j) {
-  return E == 2 ? tig + 4 * j : 2 * tig + (j & 1) + 8 * (j >> 1);
-}
+// (the token pairs a transposed ldmatrix gives the V operand)
+__device__ __forceinline__ int gq_tau(int tig, int j) { return 2 * tig + (j & 1) + 8 * (j >> 1); }
 
 // Running state of the item in progress.
 struct GqState {
   float o[8][4];   // O^T tiles: head tig, rows gid, gid + 8 of m-tile mt, columns hi / lo
   float m, m8, l;  // head tig: reference, reference + 8, sum over this lane's rows
-  uint64_t bias2;  // head gid / 2, groups 2 (gid & 1) + {0, 1}: sum over this lane's tokens of p * min
+  uint64_t bias2;  // head gid / 2, the lane's two groups: sum over its tokens of p * min
   float down, vlim;
 };
 
@@ -262,15 +264,14 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
     p[u][1] = ex2_ftz(x[u][1] - S.m);
     S.l += p[u][0] + p[u][1];
   }
-  // this lane's B' rows are tokens tau_j of head gid / 2: the V operand's
-  // token pairs, tig + 4 j for INT2, the transposed-ldmatrix order
-  // 2 tig + (j & 1) + 8 (j >> 1) otherwise
+  // this lane's B' rows are tokens tau_j = 2 tig + (j & 1) + 8 (j >> 1) of
+  // head gid / 2
   float P[SUB][4];
 #pragma unroll
   for (int u = 0; u < SUB; ++u)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int tau = gq_tau<E>(tig, j);
+      const int tau = gq_tau(tig, j);
       P[u][j] = __shfl_sync(0xffffffffu, p[u][tau >> 3], 4 * (tau & 7) + (gid >> 1));
     }
 
@@ -299,9 +300,10 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
       mma16816(S.o[mt], a[0], a[1], a[2], a[3], bb0, bb1);
     }
   } else {
-    // this lane forms both parts for groups ga, ga + 1 (ga = 2 (gid & 1)) of
-    // head gid / 2; the partner lane (lane ^ 4, the other column of the head)
-    // forms them for the other two groups
+    // the lane's two groups of head gid / 2: INT4 ga, ga + 1 (ga = 2 (gid & 1)),
+    // whose B' parts it forms for itself and for its partner lane (lane ^ 4,
+    // the other column of the head); INT2 (gid & 1) and 2 + (gid & 1), the
+    // groups of its own columns in the two B' matrices
     const int ga = 2 * (gid & 1);
     // per subtile: scales, value unit, B', value MMAs (fewer live registers)
 #pragma unroll
@@ -309,8 +311,15 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
       float vs[4][2], vm[4][2];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int row = 16 * (u0 + u) + gq_tau<E>(tig, j);
-        uint2 raw = *reinterpret_cast<const uint2*>(st + G::VSOFF + row * 16 + 4 * ga);
+        const int row = 16 * (u0 + u) + gq_tau(tig, j);
+        const unsigned char* sr = st + G::VSOFF + row * 16;
+        uint2 raw;
+        if constexpr (E == 1) {
+          raw = *reinterpret_cast<const uint2*>(sr + 4 * ga);
+        } else {
+          raw.x = *reinterpret_cast<const uint32_t*>(sr + 4 * (gid & 1));
+          raw.y = *reinterpret_cast<const uint32_t*>(sr + 8 + 4 * (gid & 1));
+        }
         if (!FULL && row >= nv) raw = make_uint2(0u, 0u);  // stale scales may not be numbers
         const float2 a = half2_bits_to_float2(raw.x), b = half2_bits_to_float2(raw.y);
         vs[j][0] = a.x; vm[j][0] = a.y;
@@ -323,7 +332,7 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
         for (int off = 1; off < 32; off <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
         const uint32_t eb = __float_as_uint(vmax) & 0x7F800000u;  // 2^k, vmax in [2^k, 2^(k+1))
         const float dn = __uint_as_float(0x7F000000u - eb);        // 2^-k
-        const float f = dn / S.down;                                // exact power of two
+        const float f = pow2_ratio(dn, S.down);                     // exact power of two
         S.down = dn;
         S.vlim = __uint_as_float(eb + 0x00800000u);                 // 2^(k+1)
 #pragma unroll
@@ -334,99 +343,85 @@ __device__ __forceinline__ void gq_sub(GqState& S, const GqQuery& Q, const unsig
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         S.bias2 = fma2(pk2(P[u][j], P[u][j]), pk2(vm[j][0], vm[j][1]), S.bias2);
-      // bb[g][pair]: B'_g rows (tau_0, tau_1) and (tau_2, tau_3)
-      uint32_t bb[4][2];
-      {
-        const uint64_t dn2 = pk2(S.down, S.down);
-        const uint64_t p01 = mul2(pk2(P[u][0], P[u][1]), dn2), p23 = mul2(pk2(P[u][2], P[u][3]), dn2);
+      const uint64_t dn2 = pk2(S.down, S.down);
+      const uint64_t p01 = mul2(pk2(P[u][0], P[u][1]), dn2), p23 = mul2(pk2(P[u][2], P[u][3]), dn2);
+      // the lane's two groups k = 0, 1: p * s (* 2^-A) of rows (tau_0, tau_1)
+      // and (tau_2, tau_3) split into fp16 high parts hi[k][pair] and
+      // remainders lo[k][pair]
+      uint32_t hi[2][2], lo[2][2];
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {  // group ga + k
-          const uint64_t w01 = mul2(p01, pk2(vs[0][k], vs[1][k]));
-          const uint64_t w23 = mul2(p23, pk2(vs[2][k], vs[3][k]));
-          const uint32_t h01 = h2_bits(__floats2half2_rn(lo2(w01), hi2(w01)));
-          const uint32_t h23 = h2_bits(__floats2half2_rn(lo2(w23), hi2(w23)));
-          const float2 f01 = half2_bits_to_float2(h01), f23 = half2_bits_to_float2(h23);
-          const uint64_t r01 = sub2(w01, pk2(f01.x, f01.y)), r23 = sub2(w23, pk2(f23.x, f23.y));
-          const uint32_t l01 = h2_bits(__floats2half2_rn(lo2(r01), hi2(r01)));
-          const uint32_t l23 = h2_bits(__floats2half2_rn(lo2(r23), hi2(r23)));
-          // this lane's column takes high parts (hl = 0) or low parts (hl = 1);
-          // the partner lane needs the other kind
-          const uint32_t own0 = hl ? l01 : h01, own1 = hl ? l23 : h23;
-          const uint32_t rcv0 = __shfl_xor_sync(0xffffffffu, hl ? h01 : l01, 4);
-          const uint32_t rcv1 = __shfl_xor_sync(0xffffffffu, hl ? h23 : l23, 4);
-          // groups 0, 1: own on even-gid lanes, received on odd ones; 2, 3 the reverse
-          bb[k][0] = hl ? rcv0 : own0;
-          bb[k][1] = hl ? rcv1 : own1;
-          bb[2 + k][0] = hl ? own0 : rcv0;
-          bb[2 + k][1] = hl ? own1 : rcv1;
-        }
+      for (int k = 0; k < 2; ++k) {
+        const uint64_t w01 = mul2(p01, pk2(vs[0][k], vs[1][k]));
+        const uint64_t w23 = mul2(p23, pk2(vs[2][k], vs[3][k]));
+        hi[k][0] = h2_bits(__floats2half2_rn(lo2(w01), hi2(w01)));
+        hi[k][1] = h2_bits(__floats2half2_rn(lo2(w23), hi2(w23)));
+        const float2 f01 = half2_bits_to_float2(hi[k][0]), f23 = half2_bits_to_float2(hi[k][1]);
+        const uint64_t r01 = sub2(w01, pk2(f01.x, f01.y)), r23 = sub2(w23, pk2(f23.x, f23.y));
+        lo[k][0] = h2_bits(__floats2half2_rn(lo2(r01), hi2(r01)));
+        lo[k][1] = h2_bits(__floats2half2_rn(lo2(r23), hi2(r23)));
       }
-      // A operand: m-tile mt covers 16 dims of group mt / 2
+      const int j8 = lane >> 3;
+      const int vr = 16 * (u0 + u) + (lane & 7) + 8 * (j8 & 1);  // ldmatrix row of this lane
       if constexpr (E == 2) {
-        // row gid (gid + 8) is dim 16 mt + gid (+ 8): one byte of each of two
-        // token rows, put side by side by a byte permute, then one mask
-        // word mt of a row: rows 0-7 in its low half (byte gid / 4), 8-15 in its high half
-        const uint32_t kA = gid >> 2, kB = 2 + (gid >> 2);
-        const uint32_t selA = kA | (kA << 4) | ((kA + 4) << 8) | ((kA + 4) << 12);
-        const uint32_t selB = kB | (kB << 4) | ((kB + 4) << 8) | ((kB + 4) << 12);
-        const uint32_t M = 0x00030003u << (2 * (gid & 3));
+        // B'_k (k = 0, 1) column (h, gp) = head h, group 2 k + gp; this lane
+        // holds column gid: its own parts.  A transposed ldmatrix of 8 token
+        // rows x one 16-byte unit (dims 64 k .. 64 k + 63, groups 2 k, 2 k + 1)
+        // gives lane (gid, tig) word gid (dims 64 k + 8 gid + 0..7, group
+        // 2 k + gid / 4) of tokens 2 tig, 2 tig + 1; m-tile 4 k + p takes
+        // crumbs p (rows gid) and p + 4 (rows gid + 8), so both of a lane's
+        // rows lie in group 2 k + gid / 4 and one of its two columns is theirs.
+        // The high and low parts go through two MMAs into one accumulator.
+        uint32_t r[4];  // (unit 0, tokens 0-7), (0, 8-15), (1, 0-7), (1, 8-15)
+        ldsm_x4_t(r, smem_addr(st + G::VOFF) + vr * 32 + 16 * int2_unit(vr, j8 >> 1));
 #pragma unroll
-        for (int hv = 0; hv < 2; ++hv) {
-          uint4 w[4];
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t x0 = r[2 * k], x1 = r[2 * k + 1], y0 = x0 >> 10, y1 = x1 >> 10;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            w[j] = *reinterpret_cast<const uint4*>(st + G::VOFF + (16 * (u0 + u) + tig + 4 * j) * 32 +
-                                                   16 * int2_unit(tig + 4 * j, hv));
-          const uint32_t w0[4] = {w[0].x, w[0].y, w[0].z, w[0].w}, w1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
-          const uint32_t w2[4] = {w[2].x, w[2].y, w[2].z, w[2].w}, w3[4] = {w[3].x, w[3].y, w[3].z, w[3].w};
-#pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const int mt = 4 * hv + mm;
-            mma16816(S.o[mt], __byte_perm(w0[mm], w1[mm], selA) & M, __byte_perm(w0[mm], w1[mm], selB) & M,
-                     __byte_perm(w2[mm], w3[mm], selA) & M, __byte_perm(w2[mm], w3[mm], selB) & M,
-                     bb[mt / 2][0], bb[mt / 2][1]);
+          for (int pp = 0; pp < 4; ++pp) {
+            const uint32_t a0 = crumb_at(x0, y0, pp), a1 = crumb_at(x0, y0, pp + 4);
+            const uint32_t a2 = crumb_at(x1, y1, pp), a3 = crumb_at(x1, y1, pp + 4);
+            mma16816(S.o[4 * k + pp], a0, a1, a2, a3, hi[k][0], hi[k][1]);
+            mma16816(S.o[4 * k + pp], a0, a1, a2, a3, lo[k][0], lo[k][1]);
           }
         }
       } else {
-        // a transposed ldmatrix of 8 token rows x one 16-byte unit (one group)
+        // B'_g column (h, hl) = head h, high (hl = 0) or low (hl = 1) part:
+        // this lane's column takes its own kind of part; the partner lane
+        // needs the other kind of the same groups
+        uint32_t bb[4][2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+            const uint32_t own = hl ? lo[k][pr] : hi[k][pr];
+            const uint32_t rcv = __shfl_xor_sync(0xffffffffu, hl ? hi[k][pr] : lo[k][pr], 4);
+            // groups 0, 1: own on even-gid lanes, received on odd ones; 2, 3 the reverse
+            bb[k][pr] = hl ? rcv : own;
+            bb[2 + k][pr] = hl ? own : rcv;
+          }
+        }
+        // a group is one 16-byte unit of a token row: a transposed ldmatrix
         // gives lane (gid, tig) 16-bit word gid (dims 4 gid .. 4 gid + 3 of
-        // the group) of tokens 2 tig (low half) and 2 tig + 1 (high half):
+        // the group) of tokens 2 tig (low half) and 2 tig + 1 (high half);
         // m-tile 2 g + sh takes nibbles 2 sh (rows gid) and 2 sh + 1 (rows
         // gid + 8) of group g, two masks per pair of tokens
-        const int j = lane >> 3;
-        const int row = 16 * (u0 + u) + (lane & 7) + 8 * (j & 1);
-        const uint32_t vrow = smem_addr(st + G::VOFF) + row * 64;
+        const uint32_t vrow = smem_addr(st + G::VOFF) + vr * 64;
 #pragma unroll
         for (int hv = 0; hv < 2; ++hv) {
           uint32_t r[4];  // (group 2 hv, tokens 0-7), (2 hv, 8-15), (2 hv + 1, 0-7), (2 hv + 1, 8-15)
-          ldsm_x4_t(r, vrow + 16 * int4_unit(row, 2 * hv + (j >> 1)));
+          ldsm_x4_t(r, vrow + 16 * int4_unit(vr, 2 * hv + (j8 >> 1)));
 #pragma unroll
           for (int gg = 0; gg < 2; ++gg) {
             const int g = 2 * hv + gg;
-            const uint32_t lo = r[2 * gg], hi = r[2 * gg + 1], lo8 = lo >> 8, hi8 = hi >> 8;
-            mma16816(S.o[2 * g], lo & 0x000F000Fu, lo & 0x00F000F0u, hi & 0x000F000Fu, hi & 0x00F000F0u,
+            const uint32_t x0 = r[2 * gg], x1 = r[2 * gg + 1], y0 = x0 >> 8, y1 = x1 >> 8;
+            mma16816(S.o[2 * g], x0 & 0x000F000Fu, x0 & 0x00F000F0u, x1 & 0x000F000Fu, x1 & 0x00F000F0u,
                      bb[g][0], bb[g][1]);
-            mma16816(S.o[2 * g + 1], lo8 & 0x000F000Fu, lo8 & 0x00F000F0u, hi8 & 0x000F000Fu,
-                     hi8 & 0x00F000F0u, bb[g][0], bb[g][1]);
+            mma16816(S.o[2 * g + 1], y0 & 0x000F000Fu, y0 & 0x00F000F0u, y1 & 0x000F000Fu,
+                     y1 & 0x00F000F0u, bb[g][0], bb[g][1]);
           }
         }
       }
     }
-  }
-}
-
-// One stage: its subtiles one after another; a full stage (TOK rows) needs
-// no row checks, a tail stage skips an empty second subtile.
-template <int E>
-__device__ __forceinline__ void gq_stage(GqState& S, const GqQuery& Q, const unsigned char* st,
-                                         int nv, int lane) {
-  if (nv == TG<E>::TOK) {
-    gq_sub<E, 0, true>(S, Q, st, nv, lane);
-    if constexpr (TG<E>::SUB == 2) gq_sub<E, 1, true>(S, Q, st, nv, lane);
-  } else {
-    gq_sub<E, 0, false>(S, Q, st, nv, lane);
-    if constexpr (TG<E>::SUB == 2)
-      if (nv > 16) gq_sub<E, 1, false>(S, Q, st, nv, lane);
   }
 }
 
@@ -442,20 +437,23 @@ __device__ __forceinline__ void gq_record(const GqState& S, int lane, int64_t w,
   float bias[4] = {0.f, 0.f, 0.f, 0.f};
   float f = 1.f;
   if constexpr (E != 0) {
-    float b0 = lo2(S.bias2), b1 = hi2(S.bias2);  // head gid / 2, groups 2 (gid & 1) + {0, 1}
+    // head gid / 2, the lane's two groups (INT4 2 (gid & 1) + {0, 1}, INT2
+    // (gid & 1) + {0, 2})
+    float b0 = lo2(S.bias2), b1 = hi2(S.bias2);
 #pragma unroll
     for (int off = 1; off < 4; off <<= 1) {
       b0 += __shfl_xor_sync(0xffffffffu, b0, off);
       b1 += __shfl_xor_sync(0xffffffffu, b1, off);
     }
-    // head tig's groups 0, 1 sit on lane 8 tig, groups 2, 3 on lane 8 tig + 4
-    bias[0] = __shfl_sync(0xffffffffu, b0, 8 * tig);
-    bias[1] = __shfl_sync(0xffffffffu, b1, 8 * tig);
-    bias[2] = __shfl_sync(0xffffffffu, b0, 8 * tig + 4);
-    bias[3] = __shfl_sync(0xffffffffu, b1, 8 * tig + 4);
-    // 2^A, the codes' 2^-24 and (INT2) this lane's position factor
-    const float pos = E == 1 ? 1.f : (float)(1 << (2 * (gid & 3)));
-    f = 16777216.0f / S.down / pos;
+    // head tig's groups sit on lanes 8 tig (gid even) and 8 tig + 4 (gid odd)
+    const float e0 = __shfl_sync(0xffffffffu, b0, 8 * tig), e1 = __shfl_sync(0xffffffffu, b1, 8 * tig);
+    const float o0 = __shfl_sync(0xffffffffu, b0, 8 * tig + 4), o1 = __shfl_sync(0xffffffffu, b1, 8 * tig + 4);
+    if constexpr (E == 1) {
+      bias[0] = e0; bias[1] = e1; bias[2] = o0; bias[3] = o1;
+    } else {
+      bias[0] = e0; bias[1] = o0; bias[2] = e1; bias[3] = o1;
+    }
+    f = pow2_ratio(16777216.0f, S.down);  // 2^A and the codes' 2^-24
   }
   float* dst = ws_acc + ((size_t)w * kG + tig) * 128;
   if constexpr (E == 1) {
@@ -469,6 +467,25 @@ __device__ __forceinline__ void gq_record(const GqState& S, int lane, int64_t w,
                       fmaf(S.o[2 * g][2] + S.o[2 * g][3], f16, bias[g]),
                       fmaf(S.o[2 * g + 1][0] + S.o[2 * g + 1][1], f, bias[g]),
                       fmaf(S.o[2 * g + 1][2] + S.o[2 * g + 1][3], f16, bias[g]));
+  } else if constexpr (E == 2) {
+    // m-tile 4 k + p: rows gid, gid + 8 are dims 64 k + 8 gid + p and
+    // 64 k + 8 gid + p + 4 (crumbs p, p + 4), group 2 k + gid / 4, whose
+    // column is 2 tig + gid / 4
+    const bool odd = gid & 4;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float bk = odd ? bias[2 * k + 1] : bias[2 * k];
+      float r[8];
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) {
+        const float* c = S.o[4 * k + pp];
+        r[pp] = fmaf(odd ? c[1] : c[0], f / crumb_scale(pp), bk);
+        r[pp + 4] = fmaf(odd ? c[3] : c[2], f / crumb_scale(pp + 4), bk);
+      }
+      float4* d4 = reinterpret_cast<float4*>(dst + 64 * k + 8 * gid);
+      d4[0] = make_float4(r[0], r[1], r[2], r[3]);
+      d4[1] = make_float4(r[4], r[5], r[6], r[7]);
+    }
   } else {
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
@@ -486,9 +503,9 @@ __device__ __forceinline__ void gq_run(const TcRun& R, int Hkv, const __half* __
   using G = TG<E>;
   const int lane = threadIdx.x & 31;
   TcStream<E> cs;
-  cs.init(R.regk, R.regv, R.soff, R.T0, R.T1, lane);
+  cs.init(ring, R.regk, R.regv, R.soff, R.T0, R.T1, lane);
 #pragma unroll 1
-  for (int s = 0; s < G::STAGES - 1; ++s) cs.issue_next(ring, lane);
+  for (int s = 0; s < G::STAGES - 1; ++s) cs.issue_next(lane);
 
   GqQuery Q;
   gq_query<E>(Q, q + ((int64_t)R.b * Hkv + R.g) * kG * 128, scale_log2, lane);
@@ -496,24 +513,39 @@ __device__ __forceinline__ void gq_run(const TcRun& R, int Hkv, const __half* __
   gq_reset(S);
   int64_t w = R.w0;
   const int item_stages = R.IT / G::TOK;  // item boundaries fall on stage boundaries
-  int left = item_stages, slot = 0;
+  int left = item_stages;
+  uint32_t soff = 0;
 
+  // whole stages; a record at every item boundary
 #pragma unroll 1
-  for (int k = 0; k < cs.nst; ++k) {
-    cs.issue_next(ring, lane);
+  for (int k = 0; k < cs.nfull; ++k) {
+    cs.issue_next(lane);
     cp_async_wait<G::STAGES - 1>();
     __syncwarp();
-    const unsigned char* st = ring + slot * G::STAGE;
-    slot = slot + 1 == G::STAGES ? 0 : slot + 1;
-    const int nv = min(G::TOK, cs.ntok - k * G::TOK);
-    gq_stage<E>(S, Q, st, nv, lane);
-    if (--left == 0 || k == cs.nst - 1) {
+    const unsigned char* st = ring + soff;
+    gq_sub<E, 0, true>(S, Q, st, G::TOK, lane);
+    if constexpr (G::SUB == 2) gq_sub<E, 1, true>(S, Q, st, G::TOK, lane);
+    soff = soff + G::STAGE == G::STAGES * G::STAGE ? 0u : soff + G::STAGE;
+    if (--left == 0) {
       gq_record<E>(S, lane, w, ws_acc, ws_ml);
       gq_reset(S);
       w += Hkv;
       left = item_stages;
     }
     __syncwarp();  // the stage is read before it is refilled
+  }
+  // the run's last item ends with a partial stage, or early at a stage boundary
+  if (cs.tail > 0) {
+    cs.issue_next(lane);
+    cp_async_wait<G::STAGES - 1>();
+    __syncwarp();
+    const unsigned char* st = ring + soff;
+    gq_sub<E, 0, false>(S, Q, st, cs.tail, lane);
+    if constexpr (G::SUB == 2)
+      if (cs.tail > 16) gq_sub<E, 1, false>(S, Q, st, cs.tail, lane);
+    gq_record<E>(S, lane, w, ws_acc, ws_ml);
+  } else if (left != item_stages) {
+    gq_record<E>(S, lane, w, ws_acc, ws_ml);
   }
   cp_async_wait<0>();
   __syncwarp();

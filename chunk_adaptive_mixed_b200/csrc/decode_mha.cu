@@ -280,7 +280,7 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
       for (int off = 1; off < 32; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
       const uint32_t eb = __float_as_uint(v) & 0x7F800000u;     // 2^k, v in [2^k, 2^(k+1))
       const float dn = __uint_as_float(0x7F000000u - eb);         // 2^-k
-      const float f = dn / S.down;                                 // exact power of two
+      const float f = pow2_ratio(dn, S.down);                      // exact power of two
       S.down = dn;
       S.vlim = __uint_as_float(eb + 0x00800000u);                  // 2^(k+1)
 #pragma unroll
@@ -391,7 +391,7 @@ __device__ __forceinline__ void tc_record(const TcState& S, int lane, int64_t w,
     // columns (2 tig, 2 tig + 1) are group tig's: a lane writes the dims of
     // group tig among its rows, with that group's sum of p * min
     bias = __shfl_sync(0xffffffffu, bias, 8 * tig);
-    const float up = 16777216.0f / S.down;  // 2^A and the codes' 2^-24
+    const float up = pow2_ratio(16777216.0f, S.down);  // 2^A and the codes' 2^-24
     if constexpr (E == 1) {
       // m-tiles 2 tig, 2 tig + 1: dims 32 tig + 4 gid + (0, 1, 2, 3), the odd
       // ones from nibbles at bit 4 (factor 16)
@@ -432,9 +432,9 @@ __device__ __forceinline__ void tc_run(const TcRun& R, int Hkv, const __half* __
   using G = TG<E>;
   const int lane = threadIdx.x & 31;
   TcStream<E> cs;
-  cs.init(R.regk, R.regv, R.soff, R.T0, R.T1, lane);
+  cs.init(ring, R.regk, R.regv, R.soff, R.T0, R.T1, lane);
 #pragma unroll 1
-  for (int s = 0; s < G::STAGES - 1; ++s) cs.issue_next(ring, lane);
+  for (int s = 0; s < G::STAGES - 1; ++s) cs.issue_next(lane);
 
   TcQuery Q;
   tc_query<E>(Q, q + ((int64_t)R.b * Hkv + R.g) * 128, scale_log2, lane);
@@ -442,27 +442,34 @@ __device__ __forceinline__ void tc_run(const TcRun& R, int Hkv, const __half* __
   tc_reset(S);
   int64_t w = R.w0;
   const int item_stages = R.IT / G::TOK;  // item boundaries fall on stage boundaries
-  int left = item_stages, slot = 0;
+  int left = item_stages;
+  uint32_t soff = 0;
 
+  // whole stages; a record at every item boundary
 #pragma unroll 1
-  for (int k = 0; k < cs.nst; ++k) {
-    cs.issue_next(ring, lane);
+  for (int k = 0; k < cs.nfull; ++k) {
+    cs.issue_next(lane);
     cp_async_wait<G::STAGES - 1>();
     __syncwarp();
-    const unsigned char* st = ring + slot * G::STAGE;
-    slot = slot + 1 == G::STAGES ? 0 : slot + 1;
-    const int nv = min(G::TOK, cs.ntok - k * G::TOK);
-    if (nv == G::TOK)
-      tc_stage<E, true>(S, Q, st, nv, lane);
-    else
-      tc_stage<E, false>(S, Q, st, nv, lane);
-    if (--left == 0 || k == cs.nst - 1) {
+    tc_stage<E, true>(S, Q, ring + soff, G::TOK, lane);
+    soff = soff + G::STAGE == G::STAGES * G::STAGE ? 0u : soff + G::STAGE;
+    if (--left == 0) {
       tc_record<E>(S, lane, w, ws_acc, ws_ml);
       tc_reset(S);
       w += Hkv;
       left = item_stages;
     }
     __syncwarp();  // the stage is read before it is refilled
+  }
+  // the run's last item ends with a partial stage, or early at a stage boundary
+  if (cs.tail > 0) {
+    cs.issue_next(lane);
+    cp_async_wait<G::STAGES - 1>();
+    __syncwarp();
+    tc_stage<E, false>(S, Q, ring + soff, cs.tail, lane);
+    tc_record<E>(S, lane, w, ws_acc, ws_ml);
+  } else if (left != item_stages) {
+    tc_record<E>(S, lane, w, ws_acc, ws_ml);
   }
   cp_async_wait<0>();
   __syncwarp();

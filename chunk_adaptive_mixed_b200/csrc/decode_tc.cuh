@@ -43,6 +43,12 @@ struct TG {  // stage geometry at head_dim 128
 };
 static_assert(TG<0>::STAGES >= 2 && TG<1>::STAGES >= 3 && TG<2>::STAGES >= 3, "ring too small");
 
+// a / b for powers of two a, b whose quotient is a normal float: the
+// exponent fields subtract (exact, and no division).
+__device__ __forceinline__ float pow2_ratio(float a, float b) {
+  return __uint_as_float(__float_as_uint(a) - __float_as_uint(b) + 0x3F800000u);
+}
+
 // In-place INT2 code pair at 2-bit position p (0..7) of both 16-bit halves:
 // c * 4^(p or p - 5) * 2^-24 each (positions 5..7 come from x >> 10).
 __device__ __forceinline__ uint32_t crumb_at(uint32_t x, uint32_t x10, int p) {
@@ -67,58 +73,80 @@ __device__ __forceinline__ int int4_unit(int row, int c) { return c ^ ((row >> 1
 // fall on eight different 16-byte bank groups.  Key rows are not swizzled.
 __device__ __forceinline__ int int2_unit(int row, int c) { return c ^ ((row >> 2) & 1); }
 
-// Copies of one stage: rows [0, nv) of the stage starting at the lane's
-// source pointers (already advanced to the stage's first row).
+// Shared-memory byte offsets, inside a stage, of the lane's copy
+// destinations: K codes, V codes (FP16: rows r, r + 2, ... at column c;
+// quantised: unit lane + 32 i of each code block, INT4 rows keeping their
+// four units XOR-swizzled (int4_unit), INT2 value rows their two
+// (int2_unit)); the scale rows are row lane of each scale block.
+template <int E>
+__device__ __forceinline__ uint32_t tc_dst_k(int lane) {
+  using G = TG<E>;
+  if constexpr (E == 0) return G::KOFF + (lane >> 4) * G::KROW + (lane & 15) * 16;
+  if constexpr (E == 1) return G::KOFF + (lane >> 2) * 64 + 16 * int4_unit(lane >> 2, lane & 3);
+  return G::KOFF + lane * 16;
+}
+template <int E>
+__device__ __forceinline__ uint32_t tc_dst_v(int lane) {
+  using G = TG<E>;
+  if constexpr (E == 0) return G::VOFF + (lane >> 4) * G::KROW + (lane & 15) * 16;
+  if constexpr (E == 1) return G::VOFF + (lane >> 2) * 64 + 16 * int4_unit(lane >> 2, lane & 3);
+  return G::VOFF + (lane >> 1) * 32 + 16 * int2_unit(lane >> 1, lane & 1);
+}
+
+// Copies of one stage into the slot at shared address sa: rows [0, nv) of
+// the stage starting at the lane's source pointers (already advanced to the
+// stage's first row).
 template <int E, bool FULL>
-__device__ __forceinline__ void tc_issue(unsigned char* st, const unsigned char* gk,
+__device__ __forceinline__ void tc_issue(uint32_t sa, uint32_t dk, uint32_t dv, const unsigned char* gk,
                                          const unsigned char* gv, const unsigned char* gks,
                                          const unsigned char* gvs, int nv, int lane) {
   using G = TG<E>;
   if constexpr (E == 0) {
     // 16 units per 256-byte row; the lane covers rows r, r + 2, ... at column c
-    const int r = lane >> 4, c = (lane & 15) * 16;
-    unsigned char* dk = st + G::KOFF + r * G::KROW + c;
-    unsigned char* dv = st + G::VOFF + r * G::KROW + c;
+    const int r = lane >> 4;
 #pragma unroll
     for (int i = 0; i < G::TOK / 2; ++i)
       if (FULL || 2 * i + r < nv) {
-        cp_async16(dk + i * 2 * G::KROW, gk + i * 2 * G::CROW);
-        cp_async16(dv + i * 2 * G::KROW, gv + i * 2 * G::CROW);
+        cp_async16s(sa + dk + i * 2 * G::KROW, gk + i * 2 * G::CROW);
+        cp_async16s(sa + dv + i * 2 * G::KROW, gv + i * 2 * G::CROW);
       }
   } else {
-    // codes: one contiguous block per array, unit lane + 32 i; INT4 rows keep
-    // their four units XOR-swizzled (int4_unit), INT2 value rows their two
-    // (int2_unit)
-    const int dl = E == 1 ? (lane >> 2) * 64 + 16 * int4_unit(lane >> 2, lane & 3) : lane * 16;
-    const int dlv = E == 1 ? dl : (lane >> 1) * 32 + 16 * int2_unit(lane >> 1, lane & 1);
 #pragma unroll
     for (int i = 0; i < G::TOK * G::CU / 32; ++i)
       if (FULL || (lane + 32 * i) / G::CU < nv) {
-        cp_async16(st + G::KOFF + dl + i * 512, gk + i * 512);
-        cp_async16(st + G::VOFF + dlv + i * 512, gv + i * 512);
+        cp_async16s(sa + dk + i * 512, gk + i * 512);
+        cp_async16s(sa + dv + i * 512, gv + i * 512);
       }
-    // scales: one 16-byte row per token, row lane
     if (FULL || lane < nv) {
-      cp_async16(st + G::KSOFF + lane * 16, gks);
-      cp_async16(st + G::VSOFF + lane * 16, gvs);
+      cp_async16s(sa + G::KSOFF + lane * 16, gks);
+      cp_async16s(sa + G::VSOFF + lane * 16, gvs);
     }
   }
   cp_async_commit();
 }
 
-// The copy stream of one run: the lane's sources advance one stage per issue.
+// The copy stream of one run: nfull whole stages, then a tail stage of
+// tail rows if tail > 0; the lane's sources advance one stage per issue and
+// the slots cycle through the ring.
 template <int E>
 struct TcStream {
   const unsigned char *gk, *gv, *gks, *gvs;
-  int ntok, nst, issued, slot;  // slot: ring slot of stage `issued`
+  uint32_t ring, dk, dv;  // ring's shared address; the lane's destination offsets
+  uint32_t soff;          // offset of the slot of stage `issued`
+  int nfull, tail, issued;
 
-  __device__ __forceinline__ void init(const unsigned char* regk, const unsigned char* regv,
-                                       uint64_t soff, int T0, int T1, int lane) {
+  __device__ __forceinline__ void init(unsigned char* ring_ptr, const unsigned char* regk,
+                                       const unsigned char* regv, uint64_t soff_scales, int T0, int T1,
+                                       int lane) {
     using G = TG<E>;
-    ntok = T1 - T0;
-    nst = (ntok + G::TOK - 1) / G::TOK;
+    const int ntok = T1 - T0;
+    nfull = ntok / G::TOK;
+    tail = ntok - nfull * G::TOK;
     issued = 0;
-    slot = 0;
+    ring = smem_addr(ring_ptr);
+    soff = 0;
+    dk = tc_dst_k<E>(lane);
+    dv = tc_dst_v<E>(lane);
     if constexpr (E == 0) {
       const int64_t row = (int64_t)T0 + (lane >> 4);
       gk = regk + row * G::CROW + (lane & 15) * 16;
@@ -127,32 +155,27 @@ struct TcStream {
     } else {
       gk = regk + (int64_t)T0 * G::CROW + lane * 16;
       gv = regv + (int64_t)T0 * G::CROW + lane * 16;
-      gks = regk + soff + ((int64_t)T0 + lane) * 16;
-      gvs = regv + soff + ((int64_t)T0 + lane) * 16;
+      gks = regk + soff_scales + ((int64_t)T0 + lane) * 16;
+      gvs = regv + soff_scales + ((int64_t)T0 + lane) * 16;
     }
   }
-  // Issues the run's next stage (or an empty group past its end) into the
-  // ring slot of stage `issued`.
-  __device__ __forceinline__ void issue_next(unsigned char* ring, int lane) {
+  // Issues the run's next stage (or an empty group past its end).
+  __device__ __forceinline__ void issue_next(int lane) {
     using G = TG<E>;
-    if (issued < nst) {
-      unsigned char* st = ring + slot * G::STAGE;
-      const int nv = min(G::TOK, ntok - issued * G::TOK);
-      if (nv == G::TOK)
-        tc_issue<E, true>(st, gk, gv, gks, gvs, nv, lane);
-      else
-        tc_issue<E, false>(st, gk, gv, gks, gvs, nv, lane);
-      gk += G::TOK * G::CROW;
-      gv += G::TOK * G::CROW;
-      if constexpr (E != 0) {
-        gks += G::TOK * 16;
-        gvs += G::TOK * 16;
-      }
-    } else {
+    if (issued < nfull)
+      tc_issue<E, true>(ring + soff, dk, dv, gk, gv, gks, gvs, G::TOK, lane);
+    else if (issued == nfull && tail > 0)
+      tc_issue<E, false>(ring + soff, dk, dv, gk, gv, gks, gvs, tail, lane);
+    else
       cp_async_commit();
+    gk += G::TOK * G::CROW;
+    gv += G::TOK * G::CROW;
+    if constexpr (E != 0) {
+      gks += G::TOK * 16;
+      gvs += G::TOK * 16;
     }
     ++issued;
-    slot = slot + 1 == G::STAGES ? 0 : slot + 1;
+    soff = soff + G::STAGE == G::STAGES * G::STAGE ? 0u : soff + G::STAGE;
   }
 };
 
