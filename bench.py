@@ -83,9 +83,13 @@ def measured_peaks():
 # workload, from an ncu capture (the command and counters are recorded under
 # profiles/), valid only for the pack kernel source (pack.cu) with this
 # SHA-256.
-PACK_TRAFFIC = {"workload": "llama2_7b_32l",
-                "sha256": "8a9960beeb72542fc97eda5327348a6f19cbddb77bc9d45c775727e1d8600141",
-                "bytes_per_launch": 2148355840 + 843005952}
+# DRAM bytes (read + write) of one full-size pack launch per workload, from
+# the ncu captures summarised in profiles/pack_kernel_*_traffic.md, with the
+# SHA-256 of the pack.cu they ran
+PACK_TRAFFIC = {
+    "llama2_7b_32l": {"sha256": "8a9960beeb72542fc97eda5327348a6f19cbddb77bc9d45c775727e1d8600141",
+                      "bytes_per_launch": 2148355840 + 843005952},
+}
 
 
 def pack_sources_sha256():
@@ -101,12 +105,11 @@ def pack_traffic(w, S, seed):
     """Measured DRAM bytes per pack launch, or None when the capture does not
     describe this kernel and workload."""
     from chunk_adaptive_mixed_b200 import workloads as W
-    if (PACK_TRAFFIC["sha256"] is None or w.name != PACK_TRAFFIC["workload"] or seed != 0
-            or w.num_seqs != W.get(w.name).num_seqs or S.router != "moqae" or S.lam
-            or not S.rs):
+    cap = PACK_TRAFFIC.get(w.name)
+    if (cap is None or seed != 0 or w.num_seqs != W.get(w.name).num_seqs or S.router != "moqae"
+            or S.lam or not S.rs):
         return None
-    return PACK_TRAFFIC["bytes_per_launch"] if pack_sources_sha256() == PACK_TRAFFIC["sha256"] \
-        else None
+    return cap["bytes_per_launch"] if pack_sources_sha256() == cap["sha256"] else None
 
 
 def peaks_all():
@@ -440,12 +443,12 @@ class Setup:
             for layer in range(w.layers):
                 Kn, Vn = self.kv_new[layer][s]
                 M.mq_grow_append_kv(self.shape, self.layout, Kn, Vn, self.packed[layer])
-                if timers and s == 0:
-                    timers["decode"][layer][0].record()
+                if timers:
+                    timers["decode"][s * w.layers + layer][0].record()
                 M.mq_decode_attn(self.shape, self.cap_lens, self.layout, self.packed[layer],
                                  self.q[layer][s], self.out[layer], self.ws)
-                if timers and s == 0:
-                    timers["decode"][layer][1].record()
+                if timers:
+                    timers["decode"][s * w.layers + layer][1].record()
             pending = self.fills[s] > 0
             if pending:
                 # route the full tails (all B tails are scored; only the full
@@ -483,16 +486,16 @@ class Setup:
                 timers["pack"][layer][1].record()
         for s in range(w.decode_steps):
             for layer in range(w.layers):
-                if timers and s == 0:
-                    timers["decode"][layer][0].record()
+                if timers:
+                    timers["decode"][s * w.layers + layer][0].record()
                 if self.shard is None:
                     M.mq_decode_attn(self.shape, self.lens, self.layout_of(layer),
                                      self.packed[layer], self.q[layer][s], self.out[layer],
                                      self.ws)
                 else:
                     self.decode_split(layer, s)
-                if timers and s == 0:
-                    timers["decode"][layer][1].record()
+                if timers:
+                    timers["decode"][s * w.layers + layer][1].record()
 
     def _route_maps(self):
         from chunk_adaptive_mixed_b200 import mqkv as M
@@ -643,8 +646,9 @@ def run_ours(args, rank, world, local_rank):
             tm = {"route": (E(enable_timing=True), E(enable_timing=True)),
                   "layout": (E(enable_timing=True), E(enable_timing=True)),
                   "pack": [(E(enable_timing=True), E(enable_timing=True)) for _ in range(w.layers)],
+                  # every decode call of the step (layers x decode steps)
                   "decode": [(E(enable_timing=True), E(enable_timing=True))
-                             for _ in range(w.layers)]}
+                             for _ in range(w.layers * w.decode_steps)]}
             if with_flush or not spans:
                 spans.append((E(enable_timing=True), E(enable_timing=True)))
                 spans[-1][0].record()
@@ -736,6 +740,7 @@ def run_ours(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": pack_bytes,
                          "avg_launch_ms": pack_avg},
             "decode_attn": {"GB/s": dec_gbs, "frac": dec_gbs / peak, "avg_ms_per_layer": dec_avg,
+                            "timed": "every decode call of every timed step (layers x decode steps)",
                             "frac_of_spec": dec_gbs / SPEC_HBM_GBS,
                             "tokens_per_s_attention_only": S.B / (dec_avg * w.layers / 1e3),
                             "algorithmic_bytes_per_layer": dec_bytes, **spread(dec_ms)},

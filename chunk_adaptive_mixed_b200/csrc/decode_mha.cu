@@ -505,17 +505,11 @@ cudaError_t launch_decode_mha(int64_t capacity_items, const unsigned char* layou
                               float* ws_acc, float2* ws_ml, unsigned int* counter, int* tab,
                               int B, int Hq, unsigned int* status, cudaStream_t stream) {
   cudaError_t e;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  static std::atomic<int> workers_cache[kTcMaxDevices];
   const size_t smem = kTcRing;
-  if ((e = cudaFuncSetAttribute(decode_mha_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem)) != cudaSuccess)
+  int64_t grid = 0;
+  if ((e = tc_workers(reinterpret_cast<const void*>(decode_mha_kernel), smem, workers_cache, &grid)) != cudaSuccess)
     return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_mha_kernel, 32, smem)) !=
-      cudaSuccess)
-    return e;
-  int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
   if (grid > capacity_items) grid = capacity_items;
   if (grid <= 0) return cudaSuccess;
   // the work order's prefix table, and the counter zeroed

@@ -15,6 +15,8 @@
 // item counts (the order's index) and zeroes the counter.
 #pragma once
 
+#include <atomic>
+
 #include "decode_ptx.cuh"
 
 namespace mqkv {
@@ -178,6 +180,35 @@ struct TcStream {
     soff = soff + G::STAGE == G::STAGES * G::STAGE ? 0u : soff + G::STAGE;
   }
 };
+
+// Worker warps (resident one-warp CTAs) of a decode kernel on the current
+// device, its dynamic shared-memory limit raised first.  Both depend only on
+// the kernel and the device, so each launcher keeps them in its own cache
+// (one slot per device) and a call pays for the queries once.
+constexpr int kTcMaxDevices = 64;
+inline cudaError_t tc_workers(const void* kern, size_t smem, std::atomic<int>* cache, int64_t* workers) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < kTcMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_acquire);
+    if (c > 0) {
+      *workers = c;
+      return cudaSuccess;
+    }
+  }
+  int sms = 0, per_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+      cudaSuccess)
+    return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32, smem)) != cudaSuccess)
+    return e;
+  const int c = sms * (per_sm > 0 ? per_sm : 1);
+  if (dev < kTcMaxDevices) cache[dev].store(c, std::memory_order_release);
+  *workers = c;
+  return cudaSuccess;
+}
 
 // A run: tokens [T0, T1) of one region, items of IT tokens, the first
 // item's record w0 (the next ones w0 + Hkv, ...).

@@ -59,3 +59,19 @@ def test_reference_arm_line_on_a_small_workload():
     assert line["ms_per_step"] <= line["projected_ms_per_full_step"] + 1e-9
     assert line["sample_wall_s"] * 1e3 >= line["ms_per_step"] * line["steps"] * 0.99
     assert np.isfinite(line["value"]) and line["value"] > 0
+
+
+def test_pack_traffic_only_for_the_captured_kernel_and_workload():
+    # roofline.traffic comes from an ncu capture of one pack.cu on one
+    # workload; any other source, workload or map setting reports null
+    class S:
+        router, lam, rs = "moqae", 0.0, True
+    for name, cap in bench.PACK_TRAFFIC.items():
+        w = W.get(name)
+        want = cap["bytes_per_launch"] if bench.pack_sources_sha256() == cap["sha256"] else None
+        assert bench.pack_traffic(w, S, 0) == want
+        assert bench.pack_traffic(w, S, 1) is None            # another seed, another map
+        S.lam = 1.0
+        assert bench.pack_traffic(w, S, 0) is None
+        S.lam = 0.0
+    assert bench.pack_traffic(W.get("tiny"), S, 0) is None
