@@ -89,6 +89,8 @@ def measured_peaks():
 PACK_TRAFFIC = {
     "llama2_7b_32l": {"sha256": "8a9960beeb72542fc97eda5327348a6f19cbddb77bc9d45c775727e1d8600141",
                       "bytes_per_launch": 2148355840 + 843005952},
+    "llama2_13b_128k": {"sha256": "8a9960beeb72542fc97eda5327348a6f19cbddb77bc9d45c775727e1d8600141",
+                        "bytes_per_launch": 2685038080 + 757476608},
 }
 
 

@@ -10,6 +10,7 @@
 #include <stdint.h>
 
 #include "mqkv.h"
+#include "mqkv_debug.h"
 
 namespace mqkv {
 
@@ -108,6 +109,9 @@ int64_t max_items_per_kv_head(const mq_shape& s, const int32_t* h_seq_lens, cons
 // per-hidden-block partial scores; finish_vote sums them, adds the bias, takes
 // the argmax and the chunk vote.
 size_t route_workspace_bytes(int64_t T, int D, int H);
+// Test hook (include/mqkv_debug.h): true once after the kernel's bit was armed.
+bool debug_take(uint32_t kernel_bit);
+
 cudaError_t launch_router_tc(const float* C, int64_t T, int D, int H, const float* W1,
                              const float* W2, const float* W3, void* workspace,
                              unsigned int* status, cudaStream_t stream, const float4** zpart_out,

@@ -20,9 +20,11 @@
 //   warp 8     allocates tensor memory and issues the MMAs (one thread).
 //   warp 9     brings the pre-split, pre-swizzled weight tiles with 1-D bulk
 //              copies.
-// Two shared-memory stages; full/empty mbarriers; tcgen05.commit frees a
-// stage when its MMAs complete.  Every wait is bounded: on timeout the kernel
-// records MQ_DEV_WAIT_TIMEOUT, stops, frees its tensor memory and returns.
+// Two shared-memory stages; per stage a full mbarrier (the producers), a
+// weight mbarrier (the bulk copies' bytes) and an empty one; tcgen05.commit
+// frees a stage when its MMAs complete.  Every wait is bounded: on timeout
+// the kernel records MQ_DEV_WAIT_TIMEOUT, stops, lets the weight copies it
+// started land, frees its tensor memory and returns.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -39,6 +41,7 @@ constexpr int kTcMmaWarp = kTcProdWarps;         // one thread issues the MMAs
 constexpr int kTcWeightWarp = kTcProdWarps + 1;  // one thread copies the weight tiles
 constexpr int kTcThreads = 32 * (kTcProdWarps + 2);
 constexpr uint32_t kTcWaitLimit = 1u << 24;
+constexpr uint32_t kTcTestWaitLimit = 1u << 12;  // under the test hook: a stop within milliseconds
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -65,8 +68,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kTcWaitLimit; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
@@ -203,7 +206,8 @@ template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1)
 router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
                  const unsigned char* __restrict__ Wp, const float* __restrict__ W3,
-                 float4* __restrict__ zpart, int nhb, unsigned int* status) {
+                 float4* __restrict__ zpart, int nhb, unsigned int* status, uint32_t wait_limit,
+                 int inject) {
   constexpr int HB = BN / 2;
   using S = TcSmem<BN>;
   extern __shared__ unsigned char smem_raw[];
@@ -213,7 +217,8 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcStages * S::STAGE);
   uint64_t* empty = full + kTcStages;
   uint64_t* done = empty + kTcStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* wfull = done + 1;  // the weight tiles' bytes, per stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + kTcStages);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
@@ -224,8 +229,9 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], kTcProd + 1);
+      mbar_init(&full[s], kTcProd);
       mbar_init(&empty[s], 1);
+      mbar_init(&wfull[s], 1);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -277,7 +283,7 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
       const int s = kt % kTcStages;
       const uint32_t ph = (kt / kTcStages) & 1;
       if (*(volatile int*)abort_flag) return false;
-      if (!mbar_wait(&empty[s], ph ^ 1)) { fail(); return false; }
+      if (!mbar_wait(&empty[s], ph ^ 1, wait_limit)) { fail(); return false; }
       unsigned char* hi = a_hi(s);
       unsigned char* lo = a_lo(s);
 #pragma unroll
@@ -295,7 +301,9 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
         *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
       }
       fence_proxy_async();  // generic-proxy stores -> visible to the tensor cores
-      mbar_arrive(&full[s]);
+      // (inject: the test hook withholds the first stage, so the MMA
+      // thread's bounded wait runs out)
+      if (!(inject && kt == 0)) mbar_arrive(&full[s]);
       return true;
     };
     load(0, buf0);
@@ -315,7 +323,10 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
         const int s = kt % kTcStages;
         const uint32_t ph = (kt / kTcStages) & 1;
         if (*(volatile int*)abort_flag) break;
-        if (!mbar_wait(&full[s], ph)) { fail(); break; }
+        if (!mbar_wait(&full[s], ph, wait_limit) || !mbar_wait(&wfull[s], ph, wait_limit)) {
+          fail();
+          break;
+        }
         tc_fence_after();
         const uint32_t ah = smem_u32(a_hi(s)), al = smem_u32(a_lo(s));
         const uint32_t bh = smem_u32(b_hi(s)), bl = smem_u32(b_lo(s));
@@ -334,16 +345,24 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   } else {
     // ---- weight tiles (one thread)
     if (lane == 0) {
+      int issued = 0;
       for (int kt = 0; kt < nkt; ++kt) {
         const int s = kt % kTcStages;
         const uint32_t ph = (kt / kTcStages) & 1;
         if (*(volatile int*)abort_flag) break;
-        if (!mbar_wait(&empty[s], ph ^ 1)) { fail(); break; }
+        if (!mbar_wait(&empty[s], ph ^ 1, wait_limit)) { fail(); break; }
         const unsigned char* src = Wp + ((size_t)(hb * nkt + kt) * 2) * S::B_BYTES;
-        mbar_arrive_expect_tx(&full[s], 2 * S::B_BYTES);
-        bulk_g2s(b_hi(s), src, S::B_BYTES, &full[s]);
-        bulk_g2s(b_lo(s), src + S::B_BYTES, S::B_BYTES, &full[s]);
+        mbar_arrive_expect_tx(&wfull[s], 2 * S::B_BYTES);
+        bulk_g2s(b_hi(s), src, S::B_BYTES, &wfull[s]);
+        bulk_g2s(b_lo(s), src + S::B_BYTES, S::B_BYTES, &wfull[s]);
+        issued = kt + 1;
       }
+      // after a stop, the copies this thread started must land before the
+      // CTA's shared memory goes away: each stage's latest one, waited on
+      // (bounded) through its own barrier
+      if (*(volatile int*)abort_flag)
+        for (int kt = max(0, issued - kTcStages); kt < issued; ++kt)
+          mbar_wait(&wfull[kt % kTcStages], (kt / kTcStages) & 1, wait_limit);
     }
     __syncwarp();
   }
@@ -354,7 +373,7 @@ router_tc_kernel(const float* __restrict__ C, int64_t T, int D, int nkt,
   // memory (the stages are free: every MMA has completed)
   if (warp < kTcProdWarps) {
     const int q4 = warp & 3, half = warp >> 2;
-    const bool ok = mbar_wait(done, 0);
+    const bool ok = mbar_wait(done, 0, wait_limit);
     if (!ok) fail();
     tc_fence_after();
     float z0 = 0.f, z1 = 0.f, z2 = 0.f;
@@ -469,6 +488,8 @@ template <int BN>
 cudaError_t launch_tc(const float* C, int64_t T, int D, int H, const float* W1, const float* W2,
                       const float* W3, unsigned char* Wp, float4* zpart, unsigned int* status,
                       cudaStream_t stream) {
+  // the test hook (mq_debug_arm_wait_timeout) applies to one launch
+  const bool inject = debug_take(MQ_DEBUG_ROUTER);
   const int nkt = (D + kTcKE - 1) / kTcKE;
   const int nhb = H / (BN / 2);
   prepack_weights_kernel<BN><<<dim3(nkt, nhb), 256, 0, stream>>>(W1, W2, D, H, nkt, Wp);
@@ -480,7 +501,9 @@ cudaError_t launch_tc(const float* C, int64_t T, int D, int H, const float* W1, 
                                   (int)smem)) != cudaSuccess)
     return err;
   const dim3 grid((unsigned)(((T + kTcBM - 1) / kTcBM) * nhb));
-  router_tc_kernel<BN><<<grid, kTcThreads, smem, stream>>>(C, T, D, nkt, Wp, W3, zpart, nhb, status);
+  router_tc_kernel<BN><<<grid, kTcThreads, smem, stream>>>(C, T, D, nkt, Wp, W3, zpart, nhb, status,
+                                                            inject ? kTcTestWaitLimit : kTcWaitLimit,
+                                                            inject ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -36,12 +36,16 @@ MQ_DEV_CAPACITY = 0x20
 MQ_GROW_OPEN = 0x1
 MQ_GROW_FULL = 0x2
 
-# names of every function include/mqkv.h declares
+# test hook targets (include/mqkv_debug.h)
+MQ_DEBUG_ROUTER = 0x1
+
+# names of every function include/*.h declares
 EXPORTS = ("mq_status_string", "mq_last_error", "mq_layout_bytes", "mq_packed_bytes_upper_bound",
            "mq_decode_workspace_bytes", "mq_route_workspace_bytes", "mq_packed_bytes", "mq_device_status", "mq_route_chunks",
            "mq_similarity_route", "mq_build_layout", "mq_pack_kv", "mq_decode_attn", "mq_decode_attn_noalloc",
            "mq_grow_sizes", "mq_grow_build_layout", "mq_grow_pack_kv", "mq_grow_commit",
-           "mq_grow_append_kv", "mq_grow_seal", "mq_decode_attn_partial", "mq_combine_partials")
+           "mq_grow_append_kv", "mq_grow_seal", "mq_decode_attn_partial", "mq_combine_partials",
+           "mq_debug_arm_wait_timeout")
 
 # size of the scratch array built into the library for mq_decode_attn_noalloc
 MQ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -210,6 +214,15 @@ def mq_device_status(clear: bool = True, stream=None) -> int:
     if st not in (MQ_OK, MQ_ERR_DEVICE_CHECK):
         _check(st, "mq_device_status")
     return int(flags.value)
+
+
+def mq_debug_arm_wait_timeout(kernels: int) -> None:
+    """Test hook: the next launch of each named kernel (MQ_DEBUG_*) stops at
+    a withheld stage through its bounded wait and sets MQ_DEV_WAIT_TIMEOUT."""
+    L = lib()
+    L.mq_debug_arm_wait_timeout.restype = ctypes.c_int
+    L.mq_debug_arm_wait_timeout.argtypes = [ctypes.c_uint32]
+    _check(L.mq_debug_arm_wait_timeout(int(kernels)), "mq_debug_arm_wait_timeout")
 
 
 # ---------------------------------------------------------------- the path

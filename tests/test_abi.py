@@ -13,8 +13,8 @@ from chunk_adaptive_mixed_b200 import build as B
 from chunk_adaptive_mixed_b200 import mqkv as M
 from oracle import oracle as O
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
-                      "mqkv.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+HEADER = os.path.join(INCLUDE, "mqkv.h")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -24,7 +24,9 @@ def built():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    # every header under include/ (the interface and its test hooks)
+    text = "".join(open(os.path.join(INCLUDE, f)).read() for f in sorted(os.listdir(INCLUDE))
+                   if f.endswith(".h"))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(mq_[a-z_]+)\s*\(", text)))
 
@@ -206,3 +208,13 @@ def test_grow_sizes_and_validation():
     # valid arguments, no device: a CUDA error, never a silent CPU path
     assert lib.mq_grow_build_layout(ctypes.byref(shp), lens.ctypes.data, 100, p, p, p, need,
                                     0) == M.MQ_ERR_CUDA
+
+
+def test_debug_hook_rejects_unknown_kernels():
+    # host only: arming makes no CUDA call, and bits outside MQ_DEBUG_* are refused
+    L = M.lib()
+    L.mq_debug_arm_wait_timeout.restype = ctypes.c_int
+    L.mq_debug_arm_wait_timeout.argtypes = [ctypes.c_uint32]
+    assert L.mq_debug_arm_wait_timeout(0x80) == M.MQ_ERR_INVALID_ARG
+    assert L.mq_debug_arm_wait_timeout(0) == M.MQ_OK
+
