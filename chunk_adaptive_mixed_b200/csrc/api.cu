@@ -130,9 +130,12 @@ ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens) {
   // dot products, softmax), about 374 byte-equivalents per query head group
   // for one query head (fitted to the single-precision decode rates: FP16
   // 5.2, INT4 2.7, INT2 1.85 TB/s), growing with the query heads that share a
-  // kv-head.  An item carries about 2^17 byte-equivalents (2^19 with four or
+  // kv-head.  An item carries about 2^18 byte-equivalents (2^19 with four or
   // more query heads per kv-head, whose per-item partial results are larger)
-  // so the partial results stay a few percent of the bytes read.  Small
+  // so the partial results, and the merge that reads them back, stay a few
+  // percent of the bytes read (measured: halving the items costs 2-3% of
+  // decode time, doubling them gains 1.6% with one query head per kv-head
+  // and nothing with four).  Small
   // problems are split finer (by powers of two, down to 32 tokens) so that
   // every worker warp of a 148-SM part gets several items.  Depends only on
   // the shape and the lengths, so size queries and layout builds agree
@@ -141,7 +144,7 @@ ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens) {
   const int qpg = s.num_q_heads / s.num_kv_heads;
   const int bpt[kNumExperts] = {2 * 2 * d, 2 * (d / 2 + d / 8), 2 * (d / 4 + d / 8)};
   const int arith = (374 * d / 128) * (2 + 3 * qpg) / 5;  // 0.4 + 0.6 * qpg of one head's
-  const int target = qpg >= 4 ? (1 << 19) : (1 << 17);
+  const int target = qpg >= 4 ? (1 << 19) : (1 << 18);
   ItemPolicy p;
   for (int e = 0; e < kNumExperts; ++e) {
     int m = (target / (bpt[e] + arith)) / 32 * 32;
