@@ -115,14 +115,19 @@ def pack_traffic(w, S, seed):
 
 
 def peaks_all():
-    """{hbm GB/s, bf16 TFLOP/s}: the measured copy bandwidth and the measured
-    bf16 GEMM burst rate (the router's MMAs are bf16)."""
+    """{hbm GB/s, bf16 TFLOP/s burst and sustained}: the measured copy
+    bandwidth and the measured bf16 GEMM rates (the router's MMAs are bf16).
+    The router runs inside a seconds-long step under the power cap, so its
+    fraction is taken against the sustained rate; the burst one is kept beside
+    it."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return {"hbm": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]), "source": "measured"}
-    return {"hbm": 6650.0, "bf16": 1590.0, "source": "fallback"}
+        burst = float(d["bf16_tflops"])
+        return {"hbm": float(d["hbm_gbs"]), "bf16": burst,
+                "bf16_sustained": float(d.get("bf16_tflops_sustained", burst)), "source": "measured"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
 def route_summary(S, route_ms, peaks):
@@ -130,15 +135,16 @@ def route_summary(S, route_ms, peaks):
     amount, unit, bound = S.route_work()
     maps = len(S.routers)
     rate = amount * maps / (route_ms / 1e3) / (1e9 if unit == "GB/s" else 1e12)
-    peak = peaks["hbm"] if bound == "hbm" else peaks["bf16"]
+    peak = peaks["hbm"] if bound == "hbm" else peaks["bf16_sustained"]
     out = {"router": S.router, "maps_per_step": maps, "avg_ms_per_step": route_ms,
            "achieved": rate, "unit": unit, "bound": bound, "peak": peak, "frac": rate / peak,
-           "peak_source": peaks["source"],
+           "peak_source": peaks["source"] + (" (sustained bf16 GEMM)" if bound == "tensor" else ""),
            "algorithmic_per_map": amount, "includes": "map kernels only (layout excluded)"}
     if bound == "tensor":
         # bf16 hi*hi + hi*lo + lo*hi: the tensor cores do 3x the algorithmic work
         out["tensor_passes"] = 3
         out["tensor_frac"] = 3 * rate / peak
+        out["tensor_frac_of_burst"] = 3 * rate / peaks["bf16"]
     return out
 
 

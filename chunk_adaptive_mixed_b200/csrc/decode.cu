@@ -1243,10 +1243,20 @@ cudaError_t launch_decode_t(int64_t max_items, int Hq, const unsigned char* layo
   const dim3 grid((unsigned)heads, (unsigned)S);
   const float* acc_c = ws_acc;
   const float2* ml_c = ws_ml;
-  cudaError_t e2 = partial ? launch_pdl(decode_combine_kernel<D, QPG, true, 8>, grid, dim3(256), 0,
-                                        stream, layout, Hq, acc_c, ml_c, out, split, done)
-                           : launch_pdl(decode_combine_kernel<D, QPG, false, 8>, grid, dim3(256), 0,
-                                        stream, layout, Hq, acc_c, ml_c, out, split, done);
+  cudaError_t e2;
+  if (avg <= 32) {
+    // few items per head: four warps, one round of loads each, and twice as
+    // many heads resident at once
+    e2 = partial ? launch_pdl(decode_combine_kernel<D, QPG, true, 4>, grid, dim3(128), 0, stream, layout,
+                              Hq, acc_c, ml_c, out, split, done)
+                 : launch_pdl(decode_combine_kernel<D, QPG, false, 4>, grid, dim3(128), 0, stream, layout,
+                              Hq, acc_c, ml_c, out, split, done);
+  } else {
+    e2 = partial ? launch_pdl(decode_combine_kernel<D, QPG, true, 8>, grid, dim3(256), 0, stream, layout,
+                              Hq, acc_c, ml_c, out, split, done)
+                 : launch_pdl(decode_combine_kernel<D, QPG, false, 8>, grid, dim3(256), 0, stream, layout,
+                              Hq, acc_c, ml_c, out, split, done);
+  }
   if (e2 != cudaSuccess) return e2;
   return cudaGetLastError();
 }
