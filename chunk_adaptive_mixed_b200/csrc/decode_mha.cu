@@ -152,11 +152,12 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
   const int g = gid >> 1;
   const bool hl = gid & 1;
 
-  // ---- scores of rows gid, gid + 8 of each subtile (two accumulator chains)
+  // ---- scores of rows gid, gid + 8 of each subtile (one accumulator chain
+  // per subtile; the two subtiles of a stage interleave)
   float sc[SUB][2];
 #pragma unroll
   for (int u = 0; u < SUB; ++u) {
-    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    float c0[4] = {0.f, 0.f, 0.f, 0.f};
     if constexpr (E == 0) {
       const int j = lane >> 3;
       const uint32_t arow = smem_addr(st + G::KOFF) + ((lane & 7) + (j & 1) * 8) * G::KROW + (j >> 1) * 16;
@@ -164,10 +165,10 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
       for (int ks = 0; ks < 8; ++ks) {
         uint32_t a[4];
         ldsm_x4(a, arow + ks * 32);
-        mma16816(ks < 4 ? c0 : c1, a[0], a[1], a[2], a[3], Q.qb[ks][0], Q.qb[ks][1]);
+        mma16816(c0, a[0], a[1], a[2], a[3], Q.qb[ks][0], Q.qb[ks][1]);
       }
-      sc[u][0] = ((c0[0] + c1[0]) + (c0[1] + c1[1])) * Q.sfac;
-      sc[u][1] = ((c0[2] + c1[2]) + (c0[3] + c1[3])) * Q.sfac;
+      sc[u][0] = (c0[0] + c0[1]) * Q.sfac;
+      sc[u][1] = (c0[2] + c0[3]) * Q.sfac;
     } else {
       const unsigned char* kr = st + G::KOFF + (16 * u + gid) * G::CROW;
       if constexpr (E == 1) {
@@ -180,7 +181,7 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
           const uint32_t x0 = r0[ks / 2], x1 = r1[ks / 2];
           const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
           const int nb = 2 * (ks % 2);
-          mma16816(ks < 4 ? c0 : c1, nib_at(x0, y0, nb), nib_at(x1, y1, nb), nib_at(x0, y0, nb + 1),
+          mma16816(c0, nib_at(x0, y0, nb), nib_at(x1, y1, nb), nib_at(x0, y0, nb + 1),
                    nib_at(x1, y1, nb + 1), Q.qb[ks][0], Q.qb[ks][1]);
         }
       } else {
@@ -192,7 +193,7 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
           const uint32_t x0 = r0[ks / 4], x1 = r1[ks / 4];
           const uint32_t y0 = x0 >> 10, y1 = x1 >> 10;
           const int p0 = 2 * (ks % 4);
-          mma16816(ks < 4 ? c0 : c1, crumb_at(x0, y0, p0), crumb_at(x1, y1, p0),
+          mma16816(c0, crumb_at(x0, y0, p0), crumb_at(x1, y1, p0),
                    crumb_at(x0, y0, p0 + 1), crumb_at(x1, y1, p0 + 1), Q.qb[ks][0], Q.qb[ks][1]);
         }
       }
@@ -201,9 +202,9 @@ __device__ __forceinline__ void tc_stage(TcState& S, const TcQuery& Q, const uns
       const uint2 k1 = *reinterpret_cast<const uint2*>(ksr + 8 * 16);
       const float2 a0 = half2_bits_to_float2(k0.x), b0 = half2_bits_to_float2(k0.y);
       const float2 a1 = half2_bits_to_float2(k1.x), b1 = half2_bits_to_float2(k1.y);
-      sc[u][0] = fmaf(fmaf(a0.x, c0[0] + c1[0], b0.x * (c0[1] + c1[1])), Q.sfac,
+      sc[u][0] = fmaf(fmaf(a0.x, c0[0], b0.x * c0[1]), Q.sfac,
                       fmaf(a0.y, Q.qsa, b0.y * Q.qsb));
-      sc[u][1] = fmaf(fmaf(a1.x, c0[2] + c1[2], b1.x * (c0[3] + c1[3])), Q.sfac,
+      sc[u][1] = fmaf(fmaf(a1.x, c0[2], b1.x * c0[3]), Q.sfac,
                       fmaf(a1.y, Q.qsa, b1.y * Q.qsb));
     }
   }
