@@ -43,12 +43,8 @@ def l2_evict(buf):
     line the L2 held is evicted (dirty ones written back now) and what stays
     is clean, so the next timed kernel reads its input from HBM and pays for
     no other data's write-backs."""
-    return buf.view(-1).view(torch_int64()).max()
-
-
-def torch_int64():
     import torch
-    return torch.int64
+    return buf.view(-1).view(torch.int64).max()
 SPEC_HBM_GBS = 8000.0   # B200 HBM3e data-sheet bandwidth (context beside the measured peak)
 
 
