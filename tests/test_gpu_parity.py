@@ -390,3 +390,27 @@ def test_decode_query_extremes(hq, hkv):
     out = gpu_decode(case, layout, packed, q.to(dev()))
     want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
     check_attention(out, want, "query extremes")
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2)])
+def test_many_short_sequences(hq, hkv):
+    # more sequences than one block of the work-order scan (256), many of
+    # them empty or shorter than a chunk: the prefix table over several
+    # blocks, sequences without items in a segment, and heads with one item
+    rng = np.random.default_rng(17 + hq)
+    lens = rng.integers(0, 90, size=600).astype(np.int32)
+    lens[::7] = 0
+    lens[5] = 1
+    case = Case(lens, hq, hkv, 128, 32, "f16")
+    K, V, q = random_kv(case, seed=51 + hq)
+    cmap = _map(case, MAPS["mixed"], seed=3)
+    layout = gpu_layout(case, cmap)
+    check_layout(case, layout.cpu().numpy(), cmap)
+    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+    ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, K.numpy(), V.numpy())
+    assert np.array_equal(packed[:pb].cpu().numpy(), ref)
+    out = gpu_decode(case, layout, packed, q.to(dev()))
+    want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
+    nz = lens > 0
+    check_attention(out[nz], want[nz], "many short sequences")
+    assert np.all(out[~nz] == 0.0)  # an empty sequence attends to nothing
