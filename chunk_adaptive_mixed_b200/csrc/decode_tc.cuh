@@ -103,25 +103,26 @@ __device__ __forceinline__ void tc_issue(uint32_t sa, uint32_t dk, uint32_t dv, 
                                          const unsigned char* gv, const unsigned char* gks,
                                          const unsigned char* gvs, int nv, int lane) {
   using G = TG<E>;
+  const uint64_t pol = l2_evict_first_policy();
   if constexpr (E == 0) {
     // 16 units per 256-byte row; the lane covers rows r, r + 2, ... at column c
     const int r = lane >> 4;
 #pragma unroll
     for (int i = 0; i < G::TOK / 2; ++i)
       if (FULL || 2 * i + r < nv) {
-        cp_async16s(sa + dk + i * 2 * G::KROW, gk + i * 2 * G::CROW);
-        cp_async16s(sa + dv + i * 2 * G::KROW, gv + i * 2 * G::CROW);
+        cp_async16h(sa + dk + i * 2 * G::KROW, gk + i * 2 * G::CROW, pol);
+        cp_async16h(sa + dv + i * 2 * G::KROW, gv + i * 2 * G::CROW, pol);
       }
   } else {
 #pragma unroll
     for (int i = 0; i < G::TOK * G::CU / 32; ++i)
       if (FULL || (lane + 32 * i) / G::CU < nv) {
-        cp_async16s(sa + dk + i * 512, gk + i * 512);
-        cp_async16s(sa + dv + i * 512, gv + i * 512);
+        cp_async16h(sa + dk + i * 512, gk + i * 512, pol);
+        cp_async16h(sa + dv + i * 512, gv + i * 512, pol);
       }
     if (FULL || lane < nv) {
-      cp_async16s(sa + G::KSOFF + lane * 16, gks);
-      cp_async16s(sa + G::VSOFF + lane * 16, gvs);
+      cp_async16h(sa + G::KSOFF + lane * 16, gks, pol);
+      cp_async16h(sa + G::VSOFF + lane * 16, gvs, pol);
     }
   }
   cp_async_commit();
