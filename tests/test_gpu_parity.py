@@ -414,3 +414,35 @@ def test_many_short_sequences(hq, hkv):
     nz = lens > 0
     check_attention(out[nz], want[nz], "many short sequences")
     assert np.all(out[~nz] == 0.0)  # an empty sequence attends to nothing
+
+
+@pytest.mark.parametrize("name", ["mha_f16_d128", "gqa4_f16_tails", "gqa8_d128", "gqa2_f32",
+                                  "mha_long", "gqa4_long"])
+def test_decode_is_deterministic(name):
+    # every work item starts from a fresh state and the merge takes the
+    # records in a fixed order, so repeated calls agree bit for bit however
+    # the warps' claims interleave (fresh, uninitialised workspaces; other
+    # work on the device between the calls)
+    long_cases = {
+        # one long sequence, few heads: many items per head, merged in slices
+        "mha_long": Case(np.array([40000], np.int32), 8, 8, 128, 256, "f16"),
+        "gqa4_long": Case(np.array([40000, 3000], np.int32), 16, 4, 128, 128, "f16"),
+    }
+    case = long_cases.get(name) or CASES[name]
+    cmap = _map(case, MAPS["mixed"], seed=11)
+    K, V, q = random_kv(case, seed=5)
+    layout = gpu_layout(case, cmap)
+    packed, pb = gpu_pack(case, layout, K.to(dev()), V.to(dev()))
+    qd = q.to(dev())
+    outs = []
+    for i in range(3):
+        noise = torch.empty(64 << 20, dtype=torch.uint8, device=dev()).fill_(i)
+        outs.append(gpu_decode(case, layout, packed, qd))
+        del noise
+    for o in outs[1:]:
+        assert np.array_equal(o.view(np.uint32), outs[0].view(np.uint32))
+    if name in long_cases:
+        ref = O.pack(case.Hkv, case.d, case.L, case.lens, cmap, K.numpy(), V.numpy())
+        assert np.array_equal(packed[:pb].cpu().numpy(), ref)
+        want = O.decode(case.Hq, case.Hkv, case.d, case.L, case.lens, cmap, ref, q.numpy())
+        check_attention(outs[0], want, name)
