@@ -1,5 +1,6 @@
 // decode_ptx.cuh — device helpers shared by the decode kernels (decode.cu,
-// decode_mha.cu): one inline-PTX wrapper per instruction (cp.async, f32x2
+// decode_mha.cu, decode_gqa.cu): one inline-PTX wrapper per instruction
+// (cp.async, with or without an L2 cache policy, createpolicy, f32x2
 // arithmetic, ex2, mma.sync, ldmatrix, movmatrix) and the work-item lookup.
 // Internal to libmqkv; not part of the ABI.
 #pragma once
