@@ -250,6 +250,29 @@ def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
     return units_per_rank * world / (ms_max / 1e3)
 
 
+def reduce_sum(x_local: float, device=None) -> float:
+    """Sum over ranks (bytes every rank moved).  A single process returns its
+    own value."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return x_local
+    t = torch.tensor([x_local], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def e2e_result(units_per_rank: float, world: int, ms_max: float, h2d_all: float, d2h_all: float,
+               steps: int, shared_batch: bool) -> dict:
+    """The end-to-end entry: whole-job tokens/s over the slowest rank's time
+    (every rank decodes the same sequences when the context is split), and the
+    bytes all ranks copied per step."""
+    value = (units_per_rank / (ms_max / 1e3) if shared_batch
+             else job_throughput(units_per_rank, world, ms_max))
+    return {"value": value, "unit": "tokens/s", "ms_per_step": ms_max, "steps": steps,
+            "h2d_bytes_per_step": int(h2d_all), "d2h_bytes_per_step": int(d2h_all)}
+
+
 # ------------------------------------------------------------------ our path
 
 class Setup:
@@ -819,7 +842,8 @@ def run_e2e(S, args, device):
     def load_layer(layer, K, V):
         K.copy_(host["K"][layer % len(host["K"])], non_blocking=True)
         V.copy_(host["V"][layer % len(host["V"])], non_blocking=True)
-    d2h = sum(o.numel() * o.element_size() for o in out_host) * w.decode_steps
+    # each layer's output after the step's last decode step
+    d2h = sum(o.numel() * o.element_size() for o in out_host)
 
     def e2e_step():
         S.C.copy_(host["C"], non_blocking=True)
@@ -843,6 +867,11 @@ def run_e2e(S, args, device):
 
     e2e_step()
     torch.cuda.synchronize()
+    world = 1
+    import torch.distributed as tdist
+    if tdist.is_available() and tdist.is_initialized():
+        world = tdist.get_world_size()
+        tdist.barrier()
     E = torch.cuda.Event
     a, b = E(enable_timing=True), E(enable_timing=True)
     a.record()
@@ -850,13 +879,13 @@ def run_e2e(S, args, device):
         e2e_step()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / args.e2e_steps
+    ms = reduce_timing(a.elapsed_time(b) / args.e2e_steps, device)
     del host
-    return {"value": S.B * w.decode_steps / (ms / 1e3), "unit": "tokens/s",
-            "ms_per_step": ms, "steps": args.e2e_steps,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "timed": "whole step including every host-to-device and device-to-host copy"
-            + ("; K/V from a two-layer pinned pool" if S.streamed else "")}
+    res = e2e_result(S.B * w.decode_steps, world, ms, reduce_sum(h2d, device),
+                     reduce_sum(d2h, device), args.e2e_steps, bool(args.context_split))
+    res["timed"] = ("whole step including every host-to-device and device-to-host copy"
+                    + ("; K/V from a two-layer pinned pool" if S.streamed else ""))
+    return res
 
 
 # ------------------------------------------------------------------ CPU oracle
