@@ -566,20 +566,9 @@ class Setup:
         return self.layouts[0 if self.rs else layer]
 
     def launches_per_step(self):
-        if self.shard is not None:   # partial decode (2) + combine (1) per layer and step
-            return (5 * len(self.routers) + self.w.layers
-                    + 3 * self.w.layers * self.w.decode_steps)
-        if self.grow:
-            w, n = self.w, self.w.decode_steps
-            fill_steps = sum(1 for f in self.fills if f)
-            return (5 + w.layers + n * (2 + 3 * w.layers)
-                    + fill_steps * (3 + w.layers))
-        # per map: weight split + router + vote (or one similarity kernel) and
-        # 2 layout kernels; one pack per layer; two decode kernels per layer
-        # and decode step
-        per_map = 3 if self.router == "similarity" else 5
-        return (per_map * len(self.routers) + self.w.layers
-                + 2 * self.w.layers * self.w.decode_steps)
+        return launches_per_step(self.w, len(self.routers), self.router,
+                                 sum(1 for f in self.fills if f) if self.grow else None,
+                                 self.shard is not None)
 
     def route_work(self):
         """Algorithmic work of one map: (amount, unit, bound).  The router is
@@ -589,6 +578,33 @@ class Setup:
         if self.router == "similarity":
             return (self.T * w.router_dim * 4 + self.B * w.router_dim * 4 + self.N, "GB/s", "hbm")
         return (4.0 * self.T * w.router_dim * w.router_hidden, "TFLOP/s", "tensor")
+
+
+def decode_kernels_per_call(w) -> int:
+    """The library's kernels in one decode call: with fp16 queries, d = 128 and
+    one or four query heads per kv-head the tensor-core decode comes with its
+    prep kernel (work-order table, counters) and the merge; the other decode
+    kernels with the merge only (a memset clears their counter)."""
+    tc = w.kv_dtype == "f16" and w.head_dim == 128 and w.num_q_heads // w.num_kv_heads in (1, 4)
+    return 3 if tc else 2
+
+
+def launches_per_step(w, n_maps: int, router: str, fill_steps=None, split: bool = False) -> int:
+    """The library's kernel launches in one step.  Per map: weight split +
+    router + vote (or one similarity kernel) and 2 layout kernels; one pack per
+    layer; one decode call per layer and decode step.  Growth (fill_steps =
+    decode steps that seal full tails): per decode step a commit (2 kernels)
+    and per layer an append before the decode call; per sealing step the
+    tails' routing (3) and one seal per layer.  A split context: a partial
+    decode call and a combine per layer and decode step."""
+    dk = decode_kernels_per_call(w)
+    if split:
+        return 5 * n_maps + w.layers + (dk + 1) * w.layers * w.decode_steps
+    if fill_steps is not None:
+        n = w.decode_steps
+        return 5 + w.layers + n * (2 + (1 + dk) * w.layers) + fill_steps * (3 + w.layers)
+    per_map = 3 if router == "similarity" else 5
+    return per_map * n_maps + w.layers + dk * w.layers * w.decode_steps
 
 
 DTYPE_DETAIL = ("router: fp32 operands, each product formed from bf16 parts (hi*hi + hi*lo + "

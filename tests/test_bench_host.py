@@ -75,3 +75,34 @@ def test_pack_traffic_only_for_the_captured_kernel_and_workload():
         assert bench.pack_traffic(w, S, 0) is None
         S.lam = 0.0
     assert bench.pack_traffic(W.get("tiny"), S, 0) is None
+
+
+def test_launch_counts_match_the_committed_launch_lists():
+    # the ncu launch lists under profiles/ count every library kernel over
+    # 1 warm-up + N timed steps plus one extra routing (prepack, router, vote,
+    # 2 layout kernels) that sizes the packed buffers
+    extra = 5
+    w13 = W.get("llama2_13b_128k")
+    assert bench.decode_kernels_per_call(w13) == 3     # prep + decode + merge
+    assert 3 * bench.launches_per_step(w13, 1, "moqae") + extra == 500
+    w7 = W.get("llama2_7b_32l")
+    assert 3 * bench.launches_per_step(w7, 1, "moqae") + extra == 404
+    wg = W.get("llama3_8b_gqa")
+    assert 2 * bench.launches_per_step(wg, 1, "moqae") + extra == 617
+    # fp32 queries (the CUDA-core decode): decode + merge
+    wt = W.get("tiny")
+    assert bench.decode_kernels_per_call(wt) == 2
+    assert bench.launches_per_step(wt, 1, "similarity") == 3 + 1 + 2
+    # a split context: partial decode call + combine per layer and step
+    assert bench.launches_per_step(w13, 1, "moqae", split=True) == 5 + 40 + 4 * 40
+
+
+def test_setup_counts_through_the_same_function():
+    # the method the bench line uses, on a stand-in with Setup's attributes
+    import types
+    w = W.get("llama3_8b_gqa")
+    s = types.SimpleNamespace(w=w, routers=[None], router="moqae", grow=False, fills=[],
+                              shard=None)
+    assert bench.Setup.launches_per_step(s) == bench.launches_per_step(w, 1, "moqae") == 306
+    s.grow, s.fills = True, [0, 3, 0, 1]
+    assert bench.Setup.launches_per_step(s) == 5 + 1 + 100 * (2 + 4) + 2 * (3 + 1)
