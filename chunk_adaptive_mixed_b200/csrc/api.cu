@@ -133,9 +133,9 @@ ItemPolicy item_policy(const mq_shape& s, const int32_t* h_seq_lens) {
   // kv-head.  An item carries about 2^18 byte-equivalents (2^19 with four or
   // more query heads per kv-head, whose per-item partial results are larger)
   // so the partial results, and the merge that reads them back, stay a few
-  // percent of the bytes read (measured: halving the items costs 2-3% of
-  // decode time, doubling them gains 1.6% with one query head per kv-head
-  // and nothing with four).  Small
+  // percent of the bytes read (measured with one query head per kv-head:
+  // 2^18 decodes 1.6% faster than 2^17 and as fast as 2^19; with four query
+  // heads, 2^20 is no faster than 2^19).  Small
   // problems are split finer (by powers of two, down to 32 tokens) so that
   // every worker warp of a 148-SM part gets several items.  Depends only on
   // the shape and the lengths, so size queries and layout builds agree
