@@ -218,3 +218,33 @@ def test_debug_hook_rejects_unknown_kernels():
     assert L.mq_debug_arm_wait_timeout(0x80) == M.MQ_ERR_INVALID_ARG
     assert L.mq_debug_arm_wait_timeout(0) == M.MQ_OK
 
+
+
+def test_headers_serve_plain_c_and_cxx_consumers(tmp_path):
+    # the boundary is a C ABI: a C99 program (pedantic, warnings as errors)
+    # includes the headers, links libmqkv and gets the binding's answers
+    import shutil
+    import subprocess
+    root = os.path.dirname(INCLUDE)
+    gcc, gxx = shutil.which("gcc"), shutil.which("g++")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(M.LIB_PATH)
+    exe = str(tmp_path / "consumer")
+    subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror", "-I", root,
+                    os.path.join(root, "tests", "abi_c", "consumer.c"), "-o", exe,
+                    "-L", libdir, "-lmqkv", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(line.split() for line in out if line and line != "ok")
+    assert "ok" in out
+    shp = M.shape(3, 32, 8, 128, 128)
+    lens = np.array([1000, 0, 4097], np.int32)
+    assert int(got["layout_bytes"]) == M.mq_layout_bytes(shp, lens)
+    assert int(got["packed_upper"]) == M.mq_packed_bytes_upper_bound(shp, lens)
+    assert int(got["decode_ws"]) == M.mq_decode_workspace_bytes(shp, lens)
+    if gxx is not None:
+        for h in sorted(os.listdir(INCLUDE)):
+            src = tmp_path / "h.cpp"
+            src.write_text(f'#include "include/{h}"\nint main() {{ return 0; }}\n')
+            subprocess.run([gxx, "-std=c++17", "-Wall", "-Wextra", "-Werror", "-I", root,
+                            "-fsyntax-only", str(src)], check=True)
