@@ -628,3 +628,39 @@ def test_decode_partial_records_merge_to_the_whole_sequence():
     z = O.decode_partial(Hq, Hkv, d, L, np.array([0], np.int32), np.zeros(0, np.uint8),
                          np.zeros(16, np.uint8), q)
     assert np.all(z[1][..., 0] == -np.inf) and np.all(z[1][..., 1] == 0) and np.all(z[0] == 0)
+
+
+# ------------------------------------------------------------ threads
+
+def test_oracle_results_do_not_depend_on_its_thread_count():
+    # every parallel loop of the oracle runs over independent outputs (tokens,
+    # chunks, (sequence, head) pairs), each summed serially in a fixed order,
+    # so the host's core count cannot change a stored or compared value
+    rng = np.random.default_rng(7)
+    lens = np.array([300, 0, 77, 513], np.int32)
+    Hq, Hkv, d, L, D, H = 8, 2, 64, 32, 48, 16
+    T = int(lens.sum())
+    C = rng.standard_normal((T, D)).astype(np.float32)
+    W1 = (rng.standard_normal((D, H)) / np.sqrt(D)).astype(np.float32)
+    W2 = (rng.standard_normal((D, H)) / np.sqrt(D)).astype(np.float32)
+    W3 = (rng.standard_normal((H, 3)) / np.sqrt(H)).astype(np.float32)
+    K = rng.standard_normal((T, Hkv, d)).astype(np.float16)
+    V = rng.standard_normal((T, Hkv, d)).astype(np.float16)
+    q = rng.standard_normal((len(lens), Hq, d)).astype(np.float16)
+
+    def run():
+        z32, _ = O.router_logits(C, W1, W2, W3)
+        cmap = O.route(lens, L, C, W1, W2, W3)[0]
+        packed = O.pack(Hkv, d, L, lens, cmap, K, V)
+        return z32, cmap, packed, O.decode(Hq, Hkv, d, L, lens, cmap, packed, q)
+
+    prev = O.num_threads()
+    try:
+        O.set_num_threads(1)
+        one = run()
+        O.set_num_threads(max(4, prev))
+        many = run()
+    finally:
+        O.set_num_threads(prev)
+    for a, b in zip(one, many):
+        assert np.array_equal(np.asarray(a).view(np.uint8), np.asarray(b).view(np.uint8))
