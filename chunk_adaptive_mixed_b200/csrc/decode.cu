@@ -725,9 +725,7 @@ struct MG {
   // quantised tiles leave the end of the warp's space to the V expansion tile
   static constexpr int RING = E == 0 ? kMmaRing : kMmaRing - kMmaTile * (128 + 8) * 2;
   static constexpr int STAGES = RING / STAGE < 8 ? RING / STAGE : 8;
-  // 16-byte copy units of one tile: K codes, V codes, K scales, V scales
-  static constexpr int CU = CROW / 16;                      // units per code row
-  static constexpr int UNITS = 2 * kMmaTile * CU + 2 * SROW;  // a tile's scales: SROW units
+  static constexpr int CU = CROW / 16;                      // 16-byte units per code row
 };
 static_assert(MG<128, 0>::STAGES >= 2 && MG<64, 0>::STAGES >= 2 && MG<128, 1>::STAGES >= 3 &&
                   MG<128, 2>::STAGES >= 3,

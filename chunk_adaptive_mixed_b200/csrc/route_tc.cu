@@ -40,6 +40,7 @@ constexpr int kTcProd = 32 * kTcProdWarps;
 constexpr int kTcMmaWarp = kTcProdWarps;         // one thread issues the MMAs
 constexpr int kTcWeightWarp = kTcProdWarps + 1;  // one thread copies the weight tiles
 constexpr int kTcThreads = 32 * (kTcProdWarps + 2);
+static_assert(kTcThreads == 32 * (kTcWeightWarp + 1), "the weight warp is the block's last warp");
 constexpr uint32_t kTcWaitLimit = 1u << 24;
 constexpr uint32_t kTcTestWaitLimit = 1u << 12;  // under the test hook: a stop within milliseconds
 
