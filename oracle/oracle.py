@@ -6,7 +6,6 @@ Every array argument is a numpy array; results come back as numpy arrays.
 fp16 data travels as numpy float16 (IEEE binary16 bit patterns).
 """
 import ctypes
-import os
 
 import numpy as np
 

@@ -14,7 +14,6 @@ import torch.distributed as tdist
 import torch.multiprocessing as mp
 
 from chunk_adaptive_mixed_b200 import context_split as CS
-from chunk_adaptive_mixed_b200 import workloads as W
 from oracle import oracle as O
 
 LENS = np.array([700, 96, 0, 31, 200], np.int32)   # chunks 11, 2, 0, 1, 4 at L = 64

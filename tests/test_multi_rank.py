@@ -7,9 +7,7 @@ time.  These tests run that plumbing with gloo on 127.0.0.1."""
 import os
 import socket
 
-import numpy as np
 import pytest
-import torch
 import torch.distributed as tdist
 import torch.multiprocessing as mp
 
