@@ -350,7 +350,9 @@ mq_status mq_pack_kv(const mq_shape* shape, const int32_t* h_seq_lens,
  *   o[b,h] = sum_t softmax_t(scale * q[b,h] · khat_t) vhat_t
  * with khat/vhat the dequantised K/V of kv-head h / (Hq/Hkv).  Work is split
  * into precision-homogeneous pieces of one segment each; a second pass merges
- * the pieces' (max, sum, accumulator) triples.
+ * the pieces' (max, sum, accumulator) triples.  The result is repeatable bit
+ * for bit: each piece is computed by one warp from a fresh state and the
+ * merge takes the pieces in a fixed order, however the warps interleave.
  *
  *   q            device [B, Hq, d], dtype q_dtype (MQ_F16 or MQ_F32)
  *   softmax_scale  <= 0 selects 1/sqrt(d)
